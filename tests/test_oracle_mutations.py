@@ -1,0 +1,152 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the
+pins of test_oracle.py catch each one."""
+
+import math
+
+import pytest
+import torch
+
+import oracle
+import oracle.moe_oracle as om
+import test_oracle as pins
+
+f64 = torch.float64
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(om, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def _sym_clamp(gate, up, limit):            # gate clamped on both sides
+    g = torch.clamp(gate, min=-limit, max=limit)
+    u = torch.clamp(up, min=-limit, max=limit)
+    return (g / (1.0 + torch.exp(-g))) * u
+
+
+def _no_up_clamp(gate, up, limit):
+    g = torch.clamp(gate, max=limit)
+    return (g / (1.0 + torch.exp(-g))) * up
+
+
+def _select_bias_on_logit(logits, bias, k, alpha, renorm):
+    b = torch.zeros(logits.shape[1], dtype=f64) if bias is None else bias.to(f64)
+    sel = om.Selection.__new__(om.Selection)
+    shifted = om._cpu64(logits) + b[None, :]
+    real = _orig_select(shifted, None, k, alpha, renorm)
+    s = om.sigmoid(om._cpu64(logits))
+    chosen = torch.gather(s, 1, real.ids)
+    if renorm:
+        chosen = chosen / chosen.sum(1, keepdim=True)
+    return om.Selection(real.ids, alpha * chosen, s, real.biased, real.gap)
+
+
+def _select_biased_weight(logits, bias, k, alpha, renorm):
+    sel = _orig_select(logits, bias, k, alpha, renorm)
+    chosen = torch.gather(sel.biased, 1, sel.ids)
+    if renorm:
+        chosen = chosen / chosen.sum(1, keepdim=True)
+    return om.Selection(sel.ids, alpha * chosen, sel.scores, sel.biased, sel.gap)
+
+
+def _select_tie_high(logits, bias, k, alpha, renorm):
+    E = logits.shape[1]
+    flipped = _orig_select(torch.flip(om._cpu64(logits), [1]),
+                           None if bias is None else torch.flip(bias, [0]), k, alpha, renorm)
+    return om.Selection(E - 1 - flipped.ids, flipped.weights, torch.flip(flipped.scores, [1]),
+                        torch.flip(flipped.biased, [1]), flipped.gap)
+
+
+def _select_renorm_after_alpha(logits, bias, k, alpha, renorm):
+    sel = _orig_select(logits, bias, k, 1.0, False)
+    w = alpha * sel.weights
+    if renorm:
+        w = w / w.sum(1, keepdim=True)
+    return om.Selection(sel.ids, w, sel.scores, sel.biased, sel.gap)
+
+
+def _dequant_hi_first(q, scale):
+    q = q.detach().cpu()
+    N, half = q.shape
+    codes = torch.stack([(q >> 4).to(f64), (q & 0xF).to(f64)], -1).reshape(N, 2 * half)
+    return (codes - 8.0) * om._cpu64(scale).repeat_interleave(128, dim=1)
+
+
+def _ffn_down_transposed(v, w_gate_up, w_down, limit):
+    I = w_down.shape[1]
+    gu = v @ w_gate_up.T
+    h = om.swiglu_clamped(gu[:, :I], gu[:, I:], limit)
+    return h @ w_down.reshape(I, -1)
+
+
+_orig_select = om.select_topk
+
+
+def _expect_fail(fn, *args):
+    with pytest.raises(AssertionError):
+        fn(*args)
+
+
+def test_symmetric_gate_clamp_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "swiglu_clamped", _sym_clamp)
+    _expect_fail(pins.test_hand_swiglu_clamp, hand)
+
+
+def test_missing_up_clamp_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "swiglu_clamped", _no_up_clamp)
+    _expect_fail(pins.test_hand_swiglu_clamp, hand)
+
+
+def test_bias_on_logit_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "select_topk", _select_bias_on_logit)
+    _expect_fail(pins.test_hand_router_scores_and_selection, hand)
+
+
+def test_biased_weight_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "select_topk", _select_biased_weight)
+    _expect_fail(pins.test_hand_router_scores_and_selection, hand)
+
+
+def test_tie_to_higher_id_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "select_topk", _select_tie_high)
+    _expect_fail(pins.test_hand_tie_goes_to_lower_id, hand)
+
+
+def test_renorm_after_alpha_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "select_topk", _select_renorm_after_alpha)
+    _expect_fail(pins.test_hand_router_scores_and_selection, hand)
+
+
+def test_nibble_order_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "dequant_int4_g128", _dequant_hi_first)
+    _expect_fail(pins.test_hand_w4a16_dequant, hand)
+
+
+def test_transposed_down_is_caught(monkeypatch):
+    _patch(monkeypatch, "expert_ffn", _ffn_down_transposed)
+    _expect_fail(pins.test_unclamped_ffn_is_textbook_swiglu)
+
+
+def test_scaled_shared_expert_is_caught(monkeypatch):
+    orig = om.moe_forward
+
+    def scaled(layer, **kw):
+        res = orig(layer, **kw)
+        res.out = res.out + (layer.cfg.alpha - 1.0) * res.shared
+        return res
+    _patch(monkeypatch, "moe_forward", scaled)
+    _expect_fail(pins.test_single_expert_layer_is_dense_sum)
+
+
+def test_dropped_shared_expert_is_caught(monkeypatch, hand):
+    orig = om.moe_forward
+
+    def dropped(layer, **kw):
+        res = orig(layer, **kw)
+        res.out = res.out - res.shared
+        return res
+    _patch(monkeypatch, "moe_forward", dropped)
+    _expect_fail(pins.test_hand_layer_output, hand)
+
+
+hand = pins.hand
