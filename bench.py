@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Routed-MoE SwiGLU layer forward benchmark (B200, sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the mid MoE layer (T=4096 tokens, hidden 2048, 64 experts,
+top_k=6, expert intermediate 1408, shared intermediate 2816, swiglu_limit 7,
+routed_scaling_factor 2.5, renormalised top-k), seeded synthetic inputs with
+random-init weights.  One step = one full layer forward (router -> permute ->
+grouped gate/up+SwiGLU -> grouped down -> combine) over T tokens.
+
+For N > 1 (torchrun, one process per GPU) every rank runs its own replica on
+its own tokens (weak scaling; the forward has no collective).  Timing: W
+untimed warm-up steps, then K steps between a barrier + synchronize, CUDA
+events on the launching stream, max over ranks.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed-MoE layer tokens/s; grouped-GEMM TFLOP/s as % of B200 bf16 dense peak"
+CONFIG_NAME = "mid"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage-iters", type=int, default=50)
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------ utilities ----
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples (50 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        self.windows = []
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def finish(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        mhz, max_mhz, reasons = [], None, set()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            if not any(a - 0.06 <= ts <= b + 0.06 for a, b in self.windows):
+                continue
+            mhz.append(sm)
+            max_mhz = smax
+            for name, v in zip(self.REASONS, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": max_mhz, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        return "GPU-" + str(u)
+    except Exception:
+        return str(dev)
+
+
+def traffic_from_profile(kernel_key: str):
+    """DRAM bytes per call of the timed FFN kernels, from the committed ncu
+    summary, only while the kernel source still matches the profiled one."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
+    if h != ent.get("source_sha256_16"):
+        return None
+    return ent["dram_bytes_per_call"]
+
+
+# ------------------------------------------------------------ workloads ----
+
+def make_inputs():
+    import moe_inputs
+    from moe_inputs.configs import CONFIGS
+    cfg = CONFIGS[CONFIG_NAME]
+    return cfg, moe_inputs.make_layer(cfg, seed=0)
+
+
+def gemm_flops(cfg):
+    R = cfg.T * cfg.k
+    routed = 6.0 * R * cfg.H * cfg.I
+    shared = 6.0 * cfg.T * cfg.H * cfg.I_s
+    return routed, shared
+
+
+def run_cpu_baseline(inp, passes=3):
+    import torch
+    import oracle
+    cores = torch.get_num_threads()
+    t0 = time.perf_counter()
+    for _ in range(passes):
+        oracle.moe_forward(inp)
+    dt = time.perf_counter() - t0
+    return {"value": passes * inp.cfg.T / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{passes} passes of the full mid layer ({inp.cfg.T} tokens each), fp64 torch CPU, "
+                      f"{dt:.1f} s"}
+
+
+def base_line(args, n_gpus, cfg):
+    return {
+        "metric": METRIC, "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+        "config": {"workload": f"{CONFIG_NAME} MoE layer: T={cfg.T} tokens/GPU, hidden={cfg.H}, E={cfg.E}, "
+                               f"top_k={cfg.k}, I={cfg.I}, I_s={cfg.I_s}, swiglu_limit={cfg.swiglu_limit}, "
+                               f"alpha={cfg.alpha}, renorm={cfg.renorm}",
+                   "tokens_per_gpu_step": cfg.T, "global_tokens_per_step": cfg.T * n_gpus,
+                   "parallelism": f"replicas x{n_gpus} (no collective in the forward)",
+                   "l2": "inputs larger than L2 (1.11 GB of expert weights streamed per step)"},
+    }
+
+
+# --------------------------------------------------------------- our arm ----
+
+def bench_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import routed_swiglu_experts_b200 as rse
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    rse.load_library()
+    cfg, inp = make_inputs()
+    c = cfg
+    layer = rse.MoELayer(hidden=c.H, num_experts=c.E, top_k=c.k, expert_inter=c.I, shared_inter=c.I_s,
+                         swiglu_limit=c.swiglu_limit, routed_scaling_factor=c.alpha, renormalize=c.renorm,
+                         router_w=inp.router_w.to(dev), correction_bias=inp.correction_bias.to(dev),
+                         w_gate_up=inp.w_gate_up.to(dev), w_down=inp.w_down.to(dev),
+                         shared_w_gate_up=inp.shared_w_gate_up.to(dev), shared_w_down=inp.shared_w_down.to(dev),
+                         max_tokens=c.T)
+    x = inp.x.to(dev)
+    out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(gpu_uuid(dev))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        layer.forward(x, out=out)
+    torch.cuda.synchronize()
+
+    # --- device-resident timing of K whole-layer steps
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    barrier()
+    clocks.mark(w0, w1)
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_per_step = ms / args.steps
+
+    # --- per-stage durations (same C-ABI calls as the forward, events between)
+    T, k, E, H = c.T, c.k, c.E, c.H
+    R = T * k
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    tw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(R, dtype=torch.int32, device=dev)
+    src = torch.empty(R, dtype=torch.int32, device=dev)
+    w_perm = torch.empty(R, dtype=torch.float32, device=dev)
+    x_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    sh = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    n_it = max(3, min(args.stage_iters, args.steps))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_it)]
+    w0 = time.time()
+    for it in range(n_it + 3):
+        ev = evs[it - 3] if it >= 3 else None
+        if ev:
+            ev[0].record(stream)
+        rse.moe_router_topk(layer.cfg, layer.w, x, T, ids, tw, layer.ws)
+        if ev:
+            ev[1].record(stream)
+        rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
+        if ev:
+            ev[2].record(stream)
+        rse.moe_grouped_swiglu_ffn(layer.cfg, layer.w, x_perm, offs, w_perm, T, y_perm, x, sh, layer.ws)
+        if ev:
+            ev[3].record(stream)
+        rse.moe_combine(layer.cfg, y_perm, row_of, None, sh, T, out)
+        if ev:
+            ev[4].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, name in enumerate(["router", "permute", "grouped_ffn", "combine"])}
+    stage_ms = {kname: max_over_ranks(v) for kname, v in stage_ms.items()}
+
+    # --- end to end through the public API with host buffers
+    x_host = inp.x.pin_memory()
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    clk = clocks.finish()
+    assert layer.device_error() == 0
+
+    peaks = measured_peaks()
+    routed_f, shared_f = gemm_flops(c)
+    ffn_s = stage_ms["grouped_ffn"] / 1e3
+    achieved = (routed_f + shared_f) / ffn_s / 1e12
+    traffic = traffic_from_profile("grouped_ffn_mid")
+    line = base_line(args, world, c)
+    line.update({
+        "value": world * c.T / (ms_per_step / 1e3), "ms_per_step": ms_per_step, "dtype": "bf16",
+        "roofline": {"kernel": "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
+                               "routed + shared expert)",
+                     "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                           if peaks.get("bf16_tflops_sustained") else None),
+                     "flops_per_call": routed_f + shared_f, "routed_flops_per_call": routed_f,
+                     "routed_tflops": routed_f / ffn_s / 1e12},
+        "stage_ms": stage_ms,
+        "e2e": {"value": world * c.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": c.T * c.H * 2, "d2h_bytes_per_step": c.T * c.H * 2},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clk,
+    })
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_cpu_baseline(inp)
+    return line
+
+
+# -------------------------------------------------------- reference arm ----
+
+def bench_reference(args):
+    """The CPU oracle, as it stands, on a bounded sample of the same layer per
+    step (the only other place bench.py runs oracle/)."""
+    import torch
+    import oracle
+    cfg, inp = make_inputs()
+    # per-step sample sized so the whole run stays within a few minutes
+    sample = 512
+    t0 = time.perf_counter()
+    oracle.moe_forward(inp, tokens=range(sample))
+    est = time.perf_counter() - t0
+    budget = 150.0
+    while sample > 16 and est * (args.steps + args.warmup) > budget:
+        sample //= 2
+        est /= 1.6
+    toks = list(range(sample))
+    for _ in range(args.warmup):
+        oracle.moe_forward(inp, tokens=toks)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_forward(inp, tokens=toks)
+    dt = time.perf_counter() - t0
+    value = args.steps * sample / dt
+    line = base_line(args, 1, cfg)
+    line.update({
+        "impl": "reference", "value": value, "ms_per_step": dt / args.steps * 1e3, "dtype": "f64",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"{sample} of the {cfg.T} tokens of the mid layer per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    })
+    return line
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(bench_reference(args)), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = bench_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

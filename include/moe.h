@@ -1,0 +1,214 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts SwiGLU
+ * layer forward: fp32 router with sigmoid scores and correction-bias top-k,
+ * token permute by expert, grouped gate/up GEMM with the clamped SwiGLU
+ * fused, grouped down GEMM with the combine weights fused, and one combine
+ * kernel that adds the shared expert.
+ *
+ * Sources for what each call computes (web pages on the method):
+ *   [glm5next] "Module glm5next_mlp" (metrale model-arch docs): §Numerics the
+ *              kernels rely on; §One all-reduce for both EP and TP; constant
+ *              KERNEL_MAX_TOP_K; modules forward, forward_prefill_gemm, build;
+ *              MOE_MODULE (token sort / permute / unpermute);
+ *              W4A16_GEMV_MODULE (routed projections outside the grouped
+ *              prefill GEMM).
+ *   [mstar]    "mstar.model.components.distributed.mlp", ParallelGatedMLP:
+ *              fused gate/up projection (gate = shard 0, up = shard 1).
+ *   [beam]     "bridge.models.beam.modeling_beam", beam_router_gating_linear
+ *              and BeamTopKRouter: router logits inp @ weight.T with both
+ *              operands in fp32.
+ *
+ * Notation: T tokens, H hidden, E routed experts, k top_k, I expert
+ * intermediate, I_s shared-expert intermediate, L swiglu_limit,
+ * alpha routed_scaling_factor, R = T*k routed rows.
+ *
+ * Conventions that hold for every call:
+ *   - Every data pointer is a DEVICE pointer (cudaMalloc / torch CUDA
+ *     memory) on the current device, unless a parameter says otherwise.
+ *     The caller owns every buffer.  The library never allocates, frees,
+ *     synchronises (except moe_read_device_error) or throws.
+ *   - All work is enqueued on `stream` (NULL = the legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-OK status means nothing was enqueued.
+ *   - Row-major layouts; bf16 is IEEE bfloat16 stored as uint16.
+ *   - Data pointers must be 16-byte aligned; H, I and I_s multiples of 8
+ *     (16-byte rows); the W4A16 format needs H and I multiples of 128.
+ *   - T == 0 returns MOE_OK and launches nothing.
+ *   - `ws` is a caller-owned device workspace of at least
+ *     moe_workspace_size(cfg, T) bytes, 256-byte aligned, whose first 256
+ *     bytes (the header) were zeroed once by moe_workspace_init.  The same
+ *     workspace serves every call below for token counts <= that T.  Calls
+ *     that share one workspace must be ordered on the GPU (same stream).
+ */
+#ifndef ROUTED_SWIGLU_EXPERTS_B200_MOE_H
+#define ROUTED_SWIGLU_EXPERTS_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size or value */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid but outside this build's limits */
+  MOE_ERR_WORKSPACE = 3,      /* workspace missing or too small */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a bounded wait inside a kernel gave up */
+} moe_status;
+
+typedef enum moe_weight_format {
+  MOE_W_BF16 = 0,        /* routed expert weights in bf16 */
+  MOE_W_INT4_G128 = 1    /* W4A16: uint4 codes, bf16 scale per 128 along K */
+} moe_weight_format;
+
+/* Largest k the router kernel selects per token ([glm5next] constant
+ * KERNEL_MAX_TOP_K: the per-token selection lives in 16-entry arrays). */
+#define MOE_MAX_TOP_K 16
+/* Largest routed expert count this build supports. */
+#define MOE_MAX_EXPERTS 1024
+
+/* Geometry and numerics of one MoE layer. */
+typedef struct moe_config {
+  int32_t hidden;                /* H  (multiple of 8) */
+  int32_t num_experts;           /* E  (1..MOE_MAX_EXPERTS); the FULL routed
+                                    count: the router ranks all experts */
+  int32_t top_k;                 /* k  (1..min(E, MOE_MAX_TOP_K)) */
+  int32_t expert_inter;          /* I  (multiple of 8) */
+  int32_t shared_inter;          /* I_s (multiple of 8; 0 = no shared expert) */
+  float swiglu_limit;            /* L > 0, required (no default); +inf = no
+                                    clamp.  gate <- min(gate, L),
+                                    up <- clamp(up, -L, L) */
+  float routed_scaling_factor;   /* alpha: multiplies the routed weights; the
+                                    shared expert is added unscaled */
+  int32_t renormalize;           /* 1: divide the k unbiased scores by their
+                                    sum before alpha; 0: no renormalisation */
+  int32_t expert_format;         /* moe_weight_format */
+} moe_config;
+
+/* Device weight handles of one layer.  Gate rows come first in every fused
+ * gate/up weight ([mstar] ParallelGatedMLP: gate = shard 0, up = shard 1). */
+typedef struct moe_weights {
+  const float* router_w;         /* fp32 [E, H] */
+  const float* correction_bias;  /* fp32 [E], or NULL for zero bias */
+  const void* w_gate_up;         /* bf16 [E, 2I, H]  | uint8 [E, 2I, H/2] */
+  const void* s_gate_up;         /* NULL             | bf16  [E, 2I, H/128] */
+  const void* w_down;            /* bf16 [E, H, I]   | uint8 [E, H, I/2] */
+  const void* s_down;            /* NULL             | bf16  [E, H, I/128] */
+  const void* shared_w_gate_up;  /* bf16 [2I_s, H] (NULL iff I_s == 0) */
+  const void* shared_w_down;     /* bf16 [H, I_s]  (NULL iff I_s == 0) */
+} moe_weights;
+/* W4A16 (int4) packing: byte q[n, c] holds the codes of k = 2c (low nibble)
+ * and k = 2c + 1 (high nibble); w[n, k] = (code - 8) * scale[n, k / 128]. */
+
+/* Human-readable name of a status.  Never NULL. */
+MOE_API const char* moe_status_string(moe_status status);
+
+/* Validate a configuration (sizes, limits, swiglu_limit not NaN and > 0).
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED. */
+MOE_API moe_status moe_config_validate(const moe_config* cfg);
+
+/* Host only.  Bytes of device workspace that every call below needs for up
+ * to `max_tokens` tokens.  *bytes is written on MOE_OK. */
+MOE_API moe_status moe_workspace_size(const moe_config* cfg, int32_t max_tokens, size_t* bytes);
+
+/* Zero the workspace header (device error word) on `stream`.  Call once
+ * after allocating a workspace. */
+MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router: logit[t, e] = sum_h x[t, h] * router_w[e, h] in fp32 ([beam]
+ * beam_router_gating_linear; no linear bias); s = sigmoid(logit); the k
+ * experts with the largest s + correction_bias, ties to the lower id
+ * ([glm5next] §Numerics: the bias steers selection only).  Selections whose
+ * fp32 biased scores are within 2^-15 of a neighbour are re-ranked from
+ * fp64 logits so the ids equal the exact-arithmetic selection.
+ *   x         bf16 [T, H]
+ *   topk_ids  int32 [T, k] out: selection order (biased desc, id asc)
+ *   topk_w    fp32  [T, k] out: alpha * s_e (renormalised first if enabled),
+ *             from the UNBIASED score. */
+MOE_API moe_status moe_router_topk(const moe_config* cfg, const moe_weights* w,
+                           const void* x, int32_t T,
+                           int32_t* topk_ids, float* topk_w,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Token sort / permute by expert ([glm5next] MOE_MODULE): a deterministic
+ * stable counting sort of the slots i = t*k + j by expert id.
+ *   topk_ids        int32 [T, k] in (each in [0, E), distinct per token)
+ *   topk_w          fp32  [T, k] in
+ *   x               bf16  [T, H] in
+ *   expert_offsets  int32 [E+1] out: expert e owns rows [off[e], off[e+1])
+ *   row_of          int32 [T*k] out: routed row of slot i
+ *   src             int32 [T*k] out: slot i of routed row r (inverse of row_of)
+ *   w_perm          fp32  [T*k] out: w_perm[row_of[i]] = topk_w[i]
+ *   x_perm          bf16  [T*k, H] out: x_perm[row_of[i]] = x[i / k]
+ * Inside an expert, rows are in ascending token order.  Ids outside [0, E)
+ * are undefined behaviour. */
+MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids,
+                       const float* topk_w, const void* x, int32_t T,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* src,
+                       float* w_perm, void* x_perm,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped expert FFN, one launch per projection for all experts
+ * ([glm5next] forward_prefill_gemm): for every routed row r of expert e,
+ *   y_perm[r] = bf16( w_perm[r] * W_down[e] h ),
+ *   h = bf16( silu(min(W_gate[e] x_perm[r], L)) * clamp(W_up[e] x_perm[r], -L, L) )
+ * ([glm5next] §Numerics: asymmetric clamp).  w_perm == NULL: unweighted.
+ * bf16 weights run on the tcgen05 tensor cores; MOE_W_INT4_G128 weights run
+ * the W4A16 kernels that dequantise in registers ([glm5next]
+ * W4A16_GEMV_MODULE).
+ * When x_shared != NULL the shared expert runs in the same launches:
+ *   shared_out[t] = bf16( SwiGLU_clamped FFN_shared(x_shared[t]) ), unscaled.
+ *   x_perm          bf16 [T*k, H]    expert_offsets int32 [E+1]
+ *   w_perm          fp32 [T*k] or NULL
+ *   y_perm          bf16 [T*k, H] out
+ *   x_shared        bf16 [T, H] or NULL;  shared_out bf16 [T, H] out */
+MOE_API moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weights* w,
+                                  const void* x_perm, const int32_t* expert_offsets,
+                                  const float* w_perm, int32_t T, void* y_perm,
+                                  const void* x_shared, void* shared_out,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine ([glm5next] §One all-reduce: shared output and routed slots are
+ * added in one combine kernel):
+ *   out[t] = bf16( shared_out[t] + sum_{j<k} c_j * y_perm[row_of[t*k + j]] )
+ * summed in fp32 in slot order, c_j = topk_w[t, j], or 1 when topk_w is
+ * NULL (y_perm already weighted).  shared_out may be NULL (no shared term).
+ *   y_perm bf16 [T*k, H]; row_of int32 [T*k]; out bf16 [T, H] (must not
+ *   alias the inputs). */
+MOE_API moe_status moe_combine(const moe_config* cfg, const void* y_perm,
+                       const int32_t* row_of, const float* topk_w,
+                       const void* shared_out, int32_t T, void* out,
+                       moe_stream_t stream);
+
+/* The whole layer in one call: router -> permute -> grouped FFN (routed +
+ * shared) -> combine, enqueued on `stream` with no host synchronisation.
+ *   x    bf16 [T, H];  out bf16 [T, H]
+ *   topk_ids_opt int32 [T, k] / topk_w_opt fp32 [T, k]: if non-NULL, the
+ *   router's selection is also written there. */
+MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
+                       const void* x, int32_t T, void* out,
+                       int32_t* topk_ids_opt, float* topk_w_opt,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace's device error
+ * word.  *code receives MOE_OK, or MOE_ERR_DEVICE_TIMEOUT if a kernel's
+ * bounded wait gave up since the last read.  Intended for tests and
+ * debugging. */
+MOE_API moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROUTED_SWIGLU_EXPERTS_B200_MOE_H */

@@ -21,7 +21,7 @@ Draw order (one ``torch.Generator`` per device):
 
 The routed/shared weights come from a generator on ``weight_device`` so the
 multi-GB layers can be drawn on the GPU in well under a second; their values
-therefore depend on that device, and every consumer of one ``MoELayer``
+therefore depend on that device, and every consumer of one ``LayerInputs``
 object (CUDA path and oracle alike) sees exactly the same tensors.
 """
 
@@ -35,12 +35,12 @@ import torch
 
 from .configs import CONFIGS, LayerConfig, SKEW_BIAS_SCALE  # noqa: F401
 
-__all__ = ["CONFIGS", "LayerConfig", "MoELayer", "make_layer", "make_x",
+__all__ = ["CONFIGS", "LayerConfig", "LayerInputs", "make_layer", "make_x",
            "zipf_log_bias", "SKEW_BIAS_SCALE"]
 
 
 @dataclasses.dataclass
-class MoELayer:
+class LayerInputs:
     """All inputs of one MoE layer call.  Shapes use T, H, E, k, I, I_s."""
     cfg: LayerConfig
     x: torch.Tensor                 # [T, H] bf16
@@ -53,7 +53,7 @@ class MoELayer:
     shared_w_gate_up: Optional[torch.Tensor]  # bf16 [2I_s, H]
     shared_w_down: Optional[torch.Tensor]     # bf16 [H, I_s]
 
-    def to(self, device) -> "MoELayer":
+    def to(self, device) -> "LayerInputs":
         def mv(t):
             return None if t is None else t.to(device)
         return dataclasses.replace(
@@ -108,7 +108,7 @@ def make_x(cfg: LayerConfig, seed: int = 0, T: Optional[int] = None):
 
 
 def make_layer(cfg: LayerConfig, seed: int = 0, weight_device="cpu",
-               T: Optional[int] = None) -> MoELayer:
+               T: Optional[int] = None) -> LayerInputs:
     """Draw one layer's inputs.  x / router / bias are always on the CPU;
     the expert and shared weights live on ``weight_device``."""
     x, router_w, bias = make_x(cfg, seed, T)
@@ -134,4 +134,4 @@ def make_layer(cfg: LayerConfig, seed: int = 0, weight_device="cpu",
         sd = _normal((H, Is), 1.0 / math.sqrt(Is), g, dev)
     else:
         sgu = sd = None
-    return MoELayer(cfg, x, router_w, bias, w_gu, w_d, s_gu, s_d, sgu, sd)
+    return LayerInputs(cfg, x, router_w, bias, w_gu, w_d, s_gu, s_d, sgu, sd)

@@ -1,0 +1,330 @@
+// The C ABI (include/moe.h): argument validation, workspace layout, and the
+// launch sequence of the layer forward.  No allocation, no host sync (except
+// moe_read_device_error), no exceptions across the boundary.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+constexpr int64_t kMaxTokens = int64_t(1) << 21;  // grid-dimension bound of the router
+
+int num_sms_current_device() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+moe_status check_tokens(const moe_config& cfg, int32_t T) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) > kMaxTokens) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config& cfg, int32_t T, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(cfg, T).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
+}
+
+int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
+
+bool is_int4(const moe_config& cfg) { return cfg.expert_format == MOE_W_INT4_G128; }
+
+moe_status check_expert_weights(const moe_config& cfg, const moe_weights* w) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (w->w_gate_up == nullptr || w->w_down == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w_gate_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
+  if (is_int4(cfg)) {
+    if (w->s_gate_up == nullptr || w->s_down == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->s_gate_up) || !aligned16(w->s_down)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+moe_status check_shared_weights(const moe_config& cfg, const moe_weights* w) {
+  if (cfg.shared_inter == 0) return MOE_OK;
+  if (w == nullptr || w->shared_w_gate_up == nullptr || w->shared_w_down == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->shared_w_gate_up) || !aligned16(w->shared_w_down)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status check_router_weights(const moe_weights* w) {
+  if (w == nullptr || w->router_w == nullptr || !aligned16(w->router_w)) return MOE_ERR_INVALID_ARG;
+  if (w->correction_bias != nullptr && (reinterpret_cast<uintptr_t>(w->correction_bias) & 3u) != 0)
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)                       \
+  do {                                      \
+    const moe_status _s = (expr);           \
+    if (_s != MOE_OK) return _s;            \
+  } while (0)
+
+#define MOE_CUDA_TRY(expr)                              \
+  do {                                                  \
+    if ((expr) != cudaSuccess) return MOE_ERR_CUDA;     \
+  } while (0)
+
+// The grouped FFN on already-permuted rows (routed) plus, optionally, the
+// shared expert on the raw tokens.
+moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_perm, const int32_t* offsets,
+                   const float* w_perm, int32_t T, void* y_perm, const void* x_shared, void* shared_out, void* ws,
+                   const WsLayout& L, cudaStream_t stream) {
+  const int H = cfg.hidden, I = cfg.expert_inter, Is = cfg.shared_inter, E = cfg.num_experts;
+  const int R = T * cfg.top_k;
+  int32_t* err = err_word(ws);
+  void* h = at<void>(ws, L.h);
+  void* hs = at<void>(ws, L.h_shared);
+  const int sms = num_sms_current_device();
+  const bool with_shared = x_shared != nullptr && Is > 0 && T > 0;
+
+  FfnProblem s_gu{}, s_d{};
+  if (with_shared) {
+    s_gu = FfnProblem{x_shared, T, nullptr, 1, w.shared_w_gate_up, Is, H, hs, nullptr};
+    s_d = FfnProblem{hs, T, nullptr, 1, w.shared_w_down, H, Is, shared_out, nullptr};
+  }
+  if (!is_int4(cfg)) {
+    FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
+    FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
+    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, with_shared ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_down(&r_d, with_shared ? &s_d : nullptr, err, sms, stream));
+  } else {
+    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, h, stream));
+    if (with_shared) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, w_perm, y_perm, stream));
+    if (with_shared) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  static std::mutex mu;
+  struct Entry { int dev; const void* func; int bytes; };
+  static Entry done[256];
+  static int ndone = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].dev == dev && done[i].func == func && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (ndone < 256) done[ndone++] = Entry{dev, func, bytes};
+  return cudaSuccess;
+}
+
+WsLayout ws_layout(const moe_config& cfg, int Tmax) {
+  WsLayout L{};
+  const size_t T = static_cast<size_t>(std::max(Tmax, 0));
+  const size_t E = cfg.num_experts, k = cfg.top_k, H = cfg.hidden, I = cfg.expert_inter, Is = cfg.shared_inter;
+  const size_t R = T * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.header = take(sizeof(WsHeader));
+  L.logits = take(router_partial_floats(static_cast<int>(T), static_cast<int>(E)) * sizeof(float));
+  L.ids = take(R * sizeof(int32_t));
+  L.wts = take(R * sizeof(float));
+  L.offsets = take((E + 1) * sizeof(int32_t));
+  L.row_of = take(R * sizeof(int32_t));
+  L.src = take(R * sizeof(int32_t));
+  L.w_perm = take(R * sizeof(float));
+  L.block_base = take(static_cast<size_t>(perm_blocks(static_cast<int>(R))) * E * sizeof(int32_t));
+  L.local_rank = take(R * sizeof(int32_t));
+  L.x_perm = take(R * H * 2);
+  L.h = take(R * I * 2);
+  L.h_shared = take(T * Is * 2);
+  L.y_perm = take(R * H * 2);
+  L.shared_out = take(T * H * 2);
+  L.total = off;
+  return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_config_validate(const moe_config* cfg) {
+  if (cfg == nullptr) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  if (c.hidden < 8 || c.hidden % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.expert_inter < 8 || c.expert_inter % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter < 0 || c.shared_inter % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts < 1) return MOE_ERR_INVALID_ARG;
+  if (c.top_k < 1 || c.top_k > c.num_experts) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (c.top_k > MOE_MAX_TOP_K) return MOE_ERR_UNSUPPORTED;
+  if (std::isnan(c.swiglu_limit) || !(c.swiglu_limit > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(c.routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  if (c.renormalize != 0 && c.renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (c.expert_format != MOE_W_BF16 && c.expert_format != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+  if (c.expert_format == MOE_W_INT4_G128 && (c.hidden % 128 != 0 || c.expert_inter % 128 != 0))
+    return MOE_ERR_UNSUPPORTED;
+  // TMA strides and boxes: rows of up to 2^31 bytes
+  if (static_cast<int64_t>(c.hidden) * 2 >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(c.expert_inter) * 2 >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_size(const moe_config* cfg, int32_t max_tokens, size_t* bytes) {
+  MOE_TRY(moe_config_validate(cfg));
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_tokens(*cfg, max_tokens));
+  *bytes = ws_layout(*cfg, max_tokens).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(ws, 0, sizeof(WsHeader), stream));
+}
+
+moe_status moe_router_topk(const moe_config* cfg, const moe_weights* w, const void* x, int32_t T, int32_t* topk_ids,
+                           float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_router_weights(w));
+  if (x == nullptr || topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(topk_ids) || !aligned16(topk_w)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  return from_cuda(launch_router(*cfg, *w, x, T, topk_ids, topk_w, at<float>(ws, L.logits), stream));
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const float* topk_w, const void* x, int32_t T,
+                       int32_t* expert_offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  const void* ptrs[] = {topk_ids, topk_w, x, expert_offsets, row_of, src, w_perm, x_perm};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  return from_cuda(launch_permute(*cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm,
+                                  at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), stream));
+}
+
+moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weights* w, const void* x_perm,
+                                  const int32_t* expert_offsets, const float* w_perm, int32_t T, void* y_perm,
+                                  const void* x_shared, void* shared_out, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_expert_weights(*cfg, w));
+  if (x_perm == nullptr || expert_offsets == nullptr || y_perm == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(expert_offsets) || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  if (w_perm != nullptr && !aligned16(w_perm)) return MOE_ERR_INVALID_ARG;
+  if (x_shared != nullptr) {
+    if (cfg->shared_inter == 0 || shared_out == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_shared) || !aligned16(shared_out)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_shared_weights(*cfg, w));
+  }
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  return run_ffn(*cfg, *w, x_perm, expert_offsets, w_perm, T, y_perm, x_shared, shared_out, ws, L, stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
+                       const void* shared_out, int32_t T, void* out, moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  if (y_perm == nullptr || row_of == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(row_of) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (topk_w != nullptr && !aligned16(topk_w)) return MOE_ERR_INVALID_ARG;
+  if (shared_out != nullptr && !aligned16(shared_out)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  return from_cuda(launch_combine(*cfg, y_perm, row_of, topk_w, shared_out, T, out, stream));
+}
+
+moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* x, int32_t T, void* out,
+                       int32_t* topk_ids_opt, float* topk_w_opt, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_router_weights(w));
+  MOE_TRY(check_expert_weights(*cfg, w));
+  MOE_TRY(check_shared_weights(*cfg, w));
+  if (x == nullptr || out == nullptr || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if ((topk_ids_opt != nullptr && !aligned16(topk_ids_opt)) || (topk_w_opt != nullptr && !aligned16(topk_w_opt)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  int32_t* ids = topk_ids_opt != nullptr ? topk_ids_opt : at<int32_t>(ws, L.ids);
+  float* wts = topk_w_opt != nullptr ? topk_w_opt : at<float>(ws, L.wts);
+  MOE_CUDA_TRY(launch_router(*cfg, *w, x, T, ids, wts, at<float>(ws, L.logits), stream));
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  float* w_perm = at<float>(ws, L.w_perm);
+  void* x_perm = at<void>(ws, L.x_perm);
+  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, at<int32_t>(ws, L.src), w_perm, x_perm,
+                              at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), stream));
+  void* y_perm = at<void>(ws, L.y_perm);
+  const bool shared = cfg->shared_inter > 0;
+  void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;
+  MOE_TRY(run_ffn(*cfg, *w, x_perm, offsets, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws, L, stream));
+  return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out, stream));
+}
+
+moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t* code) {
+  if (ws == nullptr || code == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  WsHeader h;
+  if (cudaMemcpy(&h, ws, sizeof(int32_t) * 2, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *code = h.error;
+  if (h.error != 0 && cudaMemset(ws, 0, sizeof(int32_t) * 2) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // extern "C"

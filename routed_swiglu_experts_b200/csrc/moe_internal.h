@@ -1,0 +1,75 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <algorithm>
+#include <cstddef>
+#include <cstdint>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+// Opt a kernel into `bytes` of dynamic shared memory on the current device
+// (cached per device and kernel).
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
+// Router: rows of fp32 partial logits the split-H pass may use (per expert).
+constexpr int kRouterPartialRows = 8192;
+// Near-tie width on the fp32 biased score (2^-15) below which a token's
+// selection is re-ranked from fp64 logits.
+constexpr float kRouterTieTau = 3.0517578125e-05f;
+
+struct RouterPlan {
+  int bt;           // tokens per block
+  int ks;           // splits of H
+  int k_per_split;  // H elements per split (multiple of 32)
+};
+RouterPlan router_plan(int T, int E, int H);
+size_t router_partial_floats(int Tmax, int E);
+size_t router_topk_smem(int E);
+cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const void* x, int T, int32_t* ids,
+                          float* wts, float* part, cudaStream_t stream);
+
+// Permute: slots per counting block.
+constexpr int kPermChunk = 2048;
+inline int perm_blocks(int R) { return std::max(1, (R + kPermChunk - 1) / kPermChunk); }
+cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
+                           int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
+                           int32_t* block_base, int32_t* local_rank, cudaStream_t stream);
+
+cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
+                           const void* shared_out, int T, void* out, cudaStream_t stream);
+
+// Grouped GEMMs (tcgen05).  One "problem" is a set of row groups that share
+// an A operand tensor and a weight tensor; the routed experts are one problem
+// (groups = experts, rows given by expert offsets), the shared expert another
+// (one group covering all tokens).
+struct FfnProblem {
+  const void* a;                 // bf16 [rows, K]
+  int rows;                      // total rows of a
+  const int32_t* offsets;        // [groups+1] device, or nullptr: one group of `rows`
+  int groups;
+  const void* w;                 // bf16 weights: gate/up [groups, 2N, K]; down [groups, N, K]
+  int N, K;                      // output columns, reduction length
+  void* out;                     // bf16 [rows, N]
+  const float* row_scale;        // per-row scale (down only) or nullptr
+};
+cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
+                               int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int num_sms,
+                             cudaStream_t stream);
+
+// W4A16 routed expert kernels (dequantise in registers).
+cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
+                                const int32_t* offsets, void* h, cudaStream_t stream);
+cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const void* h, const int32_t* offsets,
+                              const float* w_perm, void* y_perm, cudaStream_t stream);
+
+// Workspace layout (byte offsets from the workspace base; 256-aligned).
+struct WsLayout {
+  size_t header, logits, ids, wts, offsets, row_of, src, w_perm, block_base, local_rank;
+  size_t x_perm, h, h_shared, y_perm, shared_out, total;
+};
+WsLayout ws_layout(const moe_config& cfg, int Tmax);
+
+}  // namespace moe

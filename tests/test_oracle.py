@@ -17,7 +17,7 @@ import torch
 import torch.nn.functional as F
 
 import moe_inputs
-from moe_inputs import MoELayer
+from moe_inputs import LayerInputs
 from moe_inputs.configs import CONFIGS, LayerConfig, SKEW_BIAS_SCALE
 import oracle
 
@@ -85,7 +85,7 @@ def _hand_layer(hand, alpha=1.0, renorm=False):
     lay = hand["layer"]
     cfg = LayerConfig("hand", T=1, H=2, E=4, k=2, I=1, I_s=1, alpha=alpha, renorm=renorm)
     bf = torch.bfloat16
-    return MoELayer(cfg, torch.tensor([hand["x"]], dtype=bf),
+    return LayerInputs(cfg, torch.tensor([hand["x"]], dtype=bf),
                     torch.tensor(hand["router_w"], dtype=torch.float32),
                     torch.tensor(hand["selection"]["bias"], dtype=torch.float32),
                     torch.tensor(lay["w_gate_up"], dtype=bf), torch.tensor(lay["w_down"], dtype=bf),
@@ -225,7 +225,7 @@ def test_expert_relabel_invariance(tiny_layer, tiny_result):
     g = torch.Generator().manual_seed(7)
     pi = torch.randperm(cfg.E, generator=g)           # new id of old expert e
     inv = torch.argsort(pi)                           # old id of new expert e'
-    lay2 = MoELayer(cfg, tiny_layer.x, tiny_layer.router_w[inv], tiny_layer.correction_bias[inv],
+    lay2 = LayerInputs(cfg, tiny_layer.x, tiny_layer.router_w[inv], tiny_layer.correction_bias[inv],
                     tiny_layer.w_gate_up[inv], tiny_layer.w_down[inv], None, None,
                     tiny_layer.shared_w_gate_up, tiny_layer.shared_w_down)
     res2 = oracle.moe_forward(lay2)
@@ -301,9 +301,9 @@ def test_w4a16_layer_reduces_to_bf16_layer():
 
     qgu, sgu, wgu = pack(cfg.E, 2 * cfg.I, cfg.H)
     qd, sd, wd = pack(cfg.E, cfg.H, cfg.I)
-    lay4 = MoELayer(cfg, base.x, base.router_w, base.correction_bias, qgu, qd, sgu, sd,
+    lay4 = LayerInputs(cfg, base.x, base.router_w, base.correction_bias, qgu, qd, sgu, sd,
                     base.shared_w_gate_up, base.shared_w_down)
-    lay16 = MoELayer(cfg.with_(w4a16=False), base.x, base.router_w, base.correction_bias,
+    lay16 = LayerInputs(cfg.with_(w4a16=False), base.x, base.router_w, base.correction_bias,
                      wgu, wd, None, None, base.shared_w_gate_up, base.shared_w_down)
     a, b = oracle.moe_forward(lay4), oracle.moe_forward(lay16)
     assert (a.selection.ids == b.selection.ids).all()
