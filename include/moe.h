@@ -201,6 +201,33 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
                        int32_t* topk_ids_opt, float* topk_w_opt,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Permute without a workspace, for callers that may not allocate device
+ * memory on their enqueue path (framework / inference-server plugins and
+ * serving loops that own all device memory and only pass their own input
+ * and output buffers; allocating there can stall the device and breaks
+ * their fixed memory budget).  The method's pages have no counterpart of
+ * this call: it exists only for that deployment constraint.
+ *
+ * Same arguments, outputs and results as moe_permute, minus ws/ws_bytes.
+ * Its scratch is one fixed array inside this library
+ * (MOE_NO_ALLOC_SCRATCH_BYTES on every GPU that loads the library, held
+ * until the process exits), so:
+ *   - T * k above MOE_NO_ALLOC_MAX_ROWS returns MOE_ERR_UNSUPPORTED (use
+ *     moe_permute with a workspace for larger batches);
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing any stream;
+ *   - every call shares the array: calls whose kernels may overlap on the
+ *     GPU (other streams, other host threads) race and must be ordered on
+ *     one stream.  Nothing in it needs clearing between calls.
+ * Never calls cudaMalloc / cudaFree or any allocating routine. */
+#define MOE_NO_ALLOC_MAX_ROWS 131072
+#define MOE_NO_ALLOC_SCRATCH_BYTES 786432
+MOE_API moe_status moe_permute_no_alloc(const moe_config* cfg, const int32_t* topk_ids,
+                                        const float* topk_w, const void* x, int32_t T,
+                                        int32_t* expert_offsets, int32_t* row_of, int32_t* src,
+                                        float* w_perm, void* x_perm, moe_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the workspace's device error
  * word.  *code receives MOE_OK, or MOE_ERR_DEVICE_TIMEOUT if a kernel's
  * bounded wait gave up since the last read.  Intended for tests and

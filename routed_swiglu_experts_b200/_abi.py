@@ -31,8 +31,9 @@ MOE_MAX_EXPERTS = 1024
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",
     "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward",
-    "moe_read_device_error",
+    "moe_read_device_error", "moe_permute_no_alloc",
 )
+MOE_NO_ALLOC_MAX_ROWS = 131072
 
 
 class MoEError(RuntimeError):
@@ -94,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_combine": (ctypes.c_int, [CFG, P, P, P, P, I32, P, P]),
         "moe_forward": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, SZ, P]),
         "moe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
+        "moe_permute_no_alloc": (ctypes.c_int, [CFG, P, P, P, I32, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +195,13 @@ def moe_forward(cfg, w, x, T, out, topk_ids_opt, topk_w_opt, ws, stream=None):
     _check(load_library().moe_forward(ctypes.byref(cfg), ctypes.byref(w), _ptr(x), int(T), _ptr(out),
                                       _ptr(topk_ids_opt), _ptr(topk_w_opt), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_permute_no_alloc(cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm, stream=None):
+    """moe_permute without a workspace (scratch held inside the library)."""
+    _check(load_library().moe_permute_no_alloc(ctypes.byref(cfg), _ptr(topk_ids), _ptr(topk_w), _ptr(x), int(T),
+                                               _ptr(expert_offsets), _ptr(row_of), _ptr(src), _ptr(w_perm),
+                                               _ptr(x_perm), _stream(stream)), "moe_permute_no_alloc")
 
 
 def moe_read_device_error(ws, stream=None) -> int:

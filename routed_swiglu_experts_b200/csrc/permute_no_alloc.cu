@@ -1,0 +1,83 @@
+// moe_permute_no_alloc: the token permute for callers that cannot hand the
+// library a workspace.
+//
+// Who needs it: hosts that own every byte of device memory and only pass
+// their own input/output buffers at enqueue time -- inference-server and
+// framework plugins, and latency-critical serving loops -- are often not
+// allowed to call cudaMalloc on that path, because allocating can stall or
+// synchronise the device and breaks their fixed memory budget.  This entry
+// point takes only inputs and outputs; its scratch (per-chunk expert counts
+// and per-slot ranks) lives in one fixed device array in this library.
+//
+// The array is a file-scope __device__ symbol, so every GPU that loads the
+// library holds it (MOE_NO_ALLOC_SCRATCH_BYTES) until the process exits.
+// Host code may not use the symbol's name as a device address: the first
+// call on each device looks up the real address with cudaGetSymbolAddress
+// (with that device current) and caches it.  Every call reuses the same
+// array, so two calls whose kernels overlap on the GPU (different streams,
+// or different host threads) race on it; order them on one stream.
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kNoAllocMaxChunks = MOE_NO_ALLOC_MAX_ROWS / kPermChunk;
+constexpr size_t kNoAllocBlockBaseInts = static_cast<size_t>(kNoAllocMaxChunks) * MOE_MAX_EXPERTS;
+constexpr size_t kNoAllocScratchInts = kNoAllocBlockBaseInts + MOE_NO_ALLOC_MAX_ROWS;
+static_assert(MOE_NO_ALLOC_MAX_ROWS % kPermChunk == 0, "whole chunks");
+static_assert(kNoAllocScratchInts * sizeof(int32_t) == MOE_NO_ALLOC_SCRATCH_BYTES, "documented size");
+
+// [kNoAllocMaxChunks * E] chunk counts / bases, then [T*k] in-chunk ranks.
+// Both parts are fully written by the count kernel before anything reads
+// them, so nothing has to be cleared between calls.
+static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocScratchInts];
+
+// Device address of g_perm_scratch per device, looked up once per device.
+cudaError_t scratch_address(int32_t** out) {
+  static std::mutex mu;
+  static int32_t* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_perm_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+}  // namespace moe
+
+extern "C" MOE_API moe_status moe_permute_no_alloc(const moe_config* cfg, const int32_t* topk_ids,
+                                                   const float* topk_w, const void* x, int32_t T,
+                                                   int32_t* expert_offsets, int32_t* row_of, int32_t* src,
+                                                   float* w_perm, void* x_perm, moe_stream_t stream) {
+  using namespace moe;
+  const moe_status st = moe_config_validate(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * cfg->top_k > MOE_NO_ALLOC_MAX_ROWS) return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {topk_ids, topk_w, x, expert_offsets, row_of, src, w_perm, x_perm};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  int32_t* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* block_base = scratch;
+  int32_t* local_rank = scratch + kNoAllocBlockBaseInts;
+  const cudaError_t e = launch_permute(*cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm,
+                                       block_base, local_rank, stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
