@@ -43,6 +43,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage-iters", type=int, default=50)
+    ap.add_argument("--workload", default=CONFIG_NAME,
+                    help="layer to time (default: the mid layer the metric is quoted on)")
+    ap.add_argument("--graph", action="store_true", help="replay the forward from a captured CUDA graph")
     return ap.parse_args(argv)
 
 
@@ -141,11 +144,13 @@ def traffic_from_profile(kernel_key: str):
 
 # ------------------------------------------------------------ workloads ----
 
-def make_inputs():
+def make_inputs(name=CONFIG_NAME):
     import moe_inputs
     from moe_inputs.configs import CONFIGS
-    cfg = CONFIGS[CONFIG_NAME]
-    return cfg, moe_inputs.make_layer(cfg, seed=0)
+    cfg = CONFIGS[name]
+    # the multi-GB layers draw their weights on the GPU (same draws as the tests)
+    wdev = "cpu" if name in ("tiny", "mid") else "cuda"
+    return cfg, moe_inputs.make_layer(cfg, seed=0, weight_device=wdev)
 
 
 def gemm_flops(cfg):
@@ -168,16 +173,41 @@ def run_cpu_baseline(inp, passes=3):
                       f"{dt:.1f} s"}
 
 
+def w4a16_bytes(cfg, ids):
+    """HBM bytes one W4A16 decode call must move: codes + scales of every
+    touched expert, the bf16 shared expert, router weight, activations."""
+    touched = int(len(set(ids.reshape(-1).tolist())))
+    per_expert = (2 * cfg.I * cfg.H // 2 + cfg.H * cfg.I // 2) + 2 * (2 * cfg.I * cfg.H // 128 + cfg.H * cfg.I // 128)
+    shared = 2 * (2 * cfg.I_s * cfg.H + cfg.H * cfg.I_s)
+    router = 4 * cfg.E * cfg.H
+    acts = 2 * cfg.T * cfg.H * (2 + 2 * cfg.k)
+    return touched, touched * per_expert + shared + router + acts
+
+
+def launches_per_step(cfg):
+    """Kernels one forward launches (router 2, permute 3, combine 1, plus the
+    expert FFN path)."""
+    n = 6
+    small_shared = cfg.I_s > 0 and cfg.T <= 32 and cfg.H % 32 == 0 and cfg.I_s % 32 == 0
+    if cfg.w4a16:
+        n += 4 + (4 if small_shared else (2 if cfg.I_s > 0 else 0))
+    else:
+        n += 2 + (4 if small_shared else 0)
+    return n
+
+
 def base_line(args, n_gpus, cfg):
+    l2 = ("inputs larger than L2 (expert weights streamed per step: %.2f GB)"
+          % ((cfg.E * 3 * cfg.H * cfg.I * (0.5 if cfg.w4a16 else 2) + 6 * cfg.H * cfg.I_s) / 1e9))
     return {
         "metric": METRIC, "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
-        "config": {"workload": f"{CONFIG_NAME} MoE layer: T={cfg.T} tokens/GPU, hidden={cfg.H}, E={cfg.E}, "
+        "config": {"workload": f"{cfg.name} MoE layer: T={cfg.T} tokens/GPU, hidden={cfg.H}, E={cfg.E}, "
                                f"top_k={cfg.k}, I={cfg.I}, I_s={cfg.I_s}, swiglu_limit={cfg.swiglu_limit}, "
                                f"alpha={cfg.alpha}, renorm={cfg.renorm}",
                    "tokens_per_gpu_step": cfg.T, "global_tokens_per_step": cfg.T * n_gpus,
                    "parallelism": f"replicas x{n_gpus} (no collective in the forward)",
-                   "l2": "inputs larger than L2 (1.11 GB of expert weights streamed per step)"},
+                   "l2": l2},
     }
 
 
@@ -191,14 +221,17 @@ def bench_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     rse.load_library()
-    cfg, inp = make_inputs()
+    cfg, inp = make_inputs(args.workload)
     c = cfg
+
+    def mv(t):
+        return None if t is None else t.to(dev)
     layer = rse.MoELayer(hidden=c.H, num_experts=c.E, top_k=c.k, expert_inter=c.I, shared_inter=c.I_s,
                          swiglu_limit=c.swiglu_limit, routed_scaling_factor=c.alpha, renormalize=c.renorm,
-                         router_w=inp.router_w.to(dev), correction_bias=inp.correction_bias.to(dev),
-                         w_gate_up=inp.w_gate_up.to(dev), w_down=inp.w_down.to(dev),
-                         shared_w_gate_up=inp.shared_w_gate_up.to(dev), shared_w_down=inp.shared_w_down.to(dev),
-                         max_tokens=c.T)
+                         router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias),
+                         w_gate_up=mv(inp.w_gate_up), w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up),
+                         s_down=mv(inp.s_down), shared_w_gate_up=mv(inp.shared_w_gate_up),
+                         shared_w_down=mv(inp.shared_w_down), max_tokens=c.T)
     x = inp.x.to(dev)
     out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -218,6 +251,15 @@ def bench_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         layer.forward(x, out=out)
     torch.cuda.synchronize()
+    step = lambda: layer.forward(x, out=out)  # noqa: E731
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer.forward(x, out=out)
+        graph.replay()
+        torch.cuda.synchronize()
+        step = graph.replay
 
     # --- device-resident timing of K whole-layer steps
     barrier()
@@ -226,7 +268,7 @@ def bench_ours(args, rank, world, local_rank):
     w0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
-        layer.forward(x, out=out)
+        step()
     e1.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
@@ -300,28 +342,42 @@ def bench_ours(args, rank, world, local_rank):
     peaks = measured_peaks()
     routed_f, shared_f = gemm_flops(c)
     ffn_s = stage_ms["grouped_ffn"] / 1e3
-    achieved = (routed_f + shared_f) / ffn_s / 1e12
-    traffic = traffic_from_profile("grouped_ffn_mid")
+    if c.w4a16:
+        touched, nbytes = w4a16_bytes(c, ids.cpu())
+        achieved = nbytes / ffn_s / 1e9
+        roof = {"kernel": "W4A16 expert FFN (register-dequant gate/up+SwiGLU and down launches) + bf16 "
+                          "shared expert", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peaks['source']} HBM copy", "bytes_per_call": nbytes,
+                "touched_experts": touched}
+    else:
+        achieved = (routed_f + shared_f) / ffn_s / 1e12
+        roof = {"kernel": "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
+                          "routed + shared expert)",
+                "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": traffic_from_profile(f"grouped_ffn_{c.name}"),
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                "flops_per_call": routed_f + shared_f, "routed_flops_per_call": routed_f,
+                "routed_tflops": routed_f / ffn_s / 1e12}
     line = base_line(args, world, c)
     line.update({
         "value": world * c.T / (ms_per_step / 1e3), "ms_per_step": ms_per_step, "dtype": "bf16",
-        "roofline": {"kernel": "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
-                               "routed + shared expert)",
-                     "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                     "peak_source": f"{peaks['source']} bf16 burst",
-                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                           if peaks.get("bf16_tflops_sustained") else None),
-                     "flops_per_call": routed_f + shared_f, "routed_flops_per_call": routed_f,
-                     "routed_tflops": routed_f / ffn_s / 1e12},
+        "roofline": roof,
         "stage_ms": stage_ms,
         "e2e": {"value": world * c.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": c.T * c.H * 2, "d2h_bytes_per_step": c.T * c.H * 2},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": launches_per_step(c) * args.steps,
         "clocks": clk,
     })
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.graph:
+        line["config"]["launch"] = "CUDA graph replay of the forward"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and c.name == CONFIG_NAME:
         line["cpu_baseline"] = run_cpu_baseline(inp)
+    if graph is not None:
+        del graph
     return line
 
 
@@ -332,7 +388,7 @@ def bench_reference(args):
     step (the only other place bench.py runs oracle/)."""
     import torch
     import oracle
-    cfg, inp = make_inputs()
+    cfg, inp = make_inputs(args.workload)
     # per-step sample sized so the whole run stays within a few minutes
     sample = 512
     t0 = time.perf_counter()
@@ -354,7 +410,7 @@ def bench_reference(args):
     line.update({
         "impl": "reference", "value": value, "ms_per_step": dt / args.steps * 1e3, "dtype": "f64",
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
-                         "sample": f"{sample} of the {cfg.T} tokens of the mid layer per step"},
+                         "sample": f"{sample} of the {cfg.T} tokens of the {cfg.name} layer per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     })

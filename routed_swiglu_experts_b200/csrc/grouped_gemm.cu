@@ -5,12 +5,18 @@
 // table is the expert row offsets produced by the permute; the weights of
 // expert g are slice g of one stacked tensor, addressed by a 3-D TMA map.
 //
-// Two kernels share one persistent, warp-specialised design:
+// Three kernels share one persistent, warp-specialised design:
 //   gate/up:  h = bf16( silu(min(X Wg^T, L)) * clamp(X Wu^T, -L, L) )
 //             ("Module glm5next_mlp" §Numerics: asymmetric SwiGLU clamp;
 //              "mstar.model.components.distributed.mlp" ParallelGatedMLP:
 //              fused gate/up projection, gate = shard 0, up = shard 1)
 //   down:     y = bf16( row_scale[r] * (H Wd^T) )   (combine weight fused)
+//   router:   fp32 partial logits of x Wr^T with the fp32 router weight
+//             split exactly into three bf16 parts (hi + mid + lo) that are
+//             concatenated along K, so bf16 x bf16 products are exact and
+//             the tensor core accumulates in fp32 ("bridge.models.beam.
+//             modeling_beam" beam_router_gating_linear: fp32 operands);
+//             K is split across CTAs for small token counts.
 //
 // Tile: 128 rows x 256 accumulator columns (gate/up: 128 gate + 128 up
 // columns of the same intermediate slice; down: 256 hidden columns), K step
@@ -40,7 +46,7 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
-enum class Mode { GateUp, Down };
+enum class Mode { GateUp, Down, Router };
 
 struct alignas(64) GemmParams {
   CUtensorMap tma_a[2];
@@ -48,11 +54,17 @@ struct alignas(64) GemmParams {
   const int32_t* offsets[2];  // grouped problem: [groups+1]; else nullptr
   __nv_bfloat16* out[2];
   const float* row_scale[2];
+  float* out_f32;             // router: partial logits [k_splits, rows, n_out]
   int32_t groups[2];
   int32_t rows[2];
   int32_t n_out[2];
-  int32_t k_blocks[2];
-  int32_t n_tiles[2];
+  int32_t k_blocks[2];        // k-blocks of one pass over K (router: per part)
+  int32_t k_parts[2];         // K repetitions with different B slices (router: 3)
+  int32_t k_splits[2];        // tiles split along the (parts x k-blocks) range
+  int32_t kb_per_split[2];
+  int32_t n_tiles[2];         // output-column tiles x k_splits
+  uint32_t idesc[2];          // MMA instruction descriptor (N per problem)
+  int32_t b_bytes[2];         // bytes of one B stage
   int32_t nprob;
   float limit;
   int32_t* err;
@@ -80,6 +92,7 @@ struct TileInfo {
   int row0;     // first A row of the tile
   int nrows;    // valid rows (<= BM)
   int nidx;     // output-column tile index
+  int split;    // k-split index
 };
 
 // Tile order: problem 0 then problem 1; inside a problem, group by group;
@@ -120,7 +133,17 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams& P, const SmemC
   }
   ti.row0 = r0 + m * BM;
   ti.nrows = min(BM, r1 - ti.row0);
+  const int ks = P.k_splits[ti.p];
+  ti.split = ti.nidx % ks;
+  ti.nidx /= ks;
   return ti;
+}
+
+// k-blocks [kb0, kb1) of the (parts x k-blocks) range a tile accumulates.
+__device__ __forceinline__ void tile_k_range(const GemmParams& P, const TileInfo& ti, int& kb0, int& kb1) {
+  const int total = P.k_blocks[ti.p] * P.k_parts[ti.p];
+  kb0 = ti.split * P.kb_per_split[ti.p];
+  kb1 = min(total, kb0 + P.kb_per_split[ti.p]);
 }
 
 template <Mode MODE>
@@ -134,7 +157,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  constexpr int BN_OUT = MODE == Mode::GateUp ? 128 : 256;
+  constexpr int BN_OUT = MODE == Mode::GateUp ? 128 : 256;  // router: the problem's MMA N (<= 256)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -223,21 +246,28 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const TileInfo ti = decode_tile(P, c, t);
         const int p = ti.p;
-        const int ncol0 = ti.nidx * BN_OUT;
-        for (int kb = 0; kb < P.k_blocks[p]; ++kb) {
+        const int ncol0 = ti.nidx * (MODE == Mode::Router ? (P.b_bytes[p] / (BK * 2)) : BN_OUT);
+        int kb0, kb1;
+        tile_k_range(P, ti, kb0, kb1);
+        const uint32_t stage_tx = static_cast<uint32_t>(A_BYTES + P.b_bytes[p]);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             fail(1);
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&c.full[stage], STAGE_BYTES);
-          tma_load_2d(smem_a + stage * A_BYTES, &P.tma_a[p], kb * BK, ti.row0, &c.full[stage]);
+          const int part = kb / P.k_blocks[p];
+          const int kc = (kb - part * P.k_blocks[p]) * BK;
+          mbar_arrive_expect_tx(&c.full[stage], stage_tx);
+          tma_load_2d(smem_a + stage * A_BYTES, &P.tma_a[p], kc, ti.row0, &c.full[stage]);
           if (MODE == Mode::GateUp) {
-            tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b[p], kb * BK, ncol0, 2 * ti.g, &c.full[stage]);
-            tma_load_3d(smem_b + stage * B_BYTES + B_BYTES / 2, &P.tma_b[p], kb * BK, ncol0, 2 * ti.g + 1,
+            tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b[p], kc, ncol0, 2 * ti.g, &c.full[stage]);
+            tma_load_3d(smem_b + stage * B_BYTES + B_BYTES / 2, &P.tma_b[p], kc, ncol0, 2 * ti.g + 1,
                         &c.full[stage]);
+          } else if (MODE == Mode::Down) {
+            tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b[p], kc, ncol0, ti.g, &c.full[stage]);
           } else {
-            tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b[p], kb * BK, ncol0, ti.g, &c.full[stage]);
+            tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b[p], kc, ncol0, part, &c.full[stage]);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -259,21 +289,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   } else if (warp == 5) {
     // -------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(BM, MMA_N);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const int p = t >= c.tiles[0] ? 1 : 0;
+        const TileInfo ti = decode_tile(P, c, t);
+        const int p = ti.p;
+        const uint32_t idesc = P.idesc[p];
+        int kb0, kb1;
+        tile_k_range(P, ti, kb0, kb1);
         if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
           fail(2);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
-        for (int kb = 0; kb < P.k_blocks[p]; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
             fail(3);
             ok = false;
@@ -286,7 +319,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
             const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&c.empty[stage]);
           if (++stage == STAGES) {
@@ -315,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const TileInfo ti = decode_tile(P, c, t);
       const int p = ti.p;
-      const int ncol0 = ti.nidx * BN_OUT;
+      const int ncol0 = ti.nidx * (MODE == Mode::Router ? (P.b_bytes[p] / (BK * 2)) : BN_OUT);
       // every lane waits; the outcome is made warp-uniform before the
       // warp-collective TMEM loads
       const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
@@ -364,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
           }
         }
-      } else {
+      } else if (MODE == Mode::Down) {
         const float* rs = P.row_scale[p];
         const float scale = (rs != nullptr && row_ok) ? rs[ti.row0 + row_in_tile] : 1.f;
 #pragma unroll 1
@@ -388,6 +421,36 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
               if (col + 8 * q < N)
                 *reinterpret_cast<uint4*>(orow + col + 8 * q) =
                     make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          }
+        }
+      } else {
+        // router: fp32 partial logits of this k-split
+        const int n_mma = P.b_bytes[p] / (BK * 2);
+        const int nch = (n_mma + 31) / 32;
+        float* frow = P.out_f32 + (static_cast<size_t>(ti.split) * P.rows[p] + ti.row0 + (row_ok ? row_in_tile : 0)) * N;
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + ch * 32, v);
+          tmem_ld_wait();
+          if (ch == nch - 1) {
+            tc_fence_before();
+            mbar_arrive(&c.tmem_empty[acc]);
+          }
+          const int col = ncol0 + ch * 32;
+          if (row_ok) {
+            if ((N & 3) == 0) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (col + 4 * q < N)
+                  *reinterpret_cast<uint4*>(frow + col + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                                                             v[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 32; ++q)
+                if (col + q < N) frow[col + q] = __uint_as_float(v[q]);
+            }
           }
         }
       }
@@ -477,7 +540,12 @@ cudaError_t launch_impl(const FfnProblem* routed, const FfnProblem* shared, floa
     P.rows[i] = f.rows;
     P.n_out[i] = f.N;
     P.k_blocks[i] = (f.K + BK - 1) / BK;
+    P.k_parts[i] = 1;
+    P.k_splits[i] = 1;
+    P.kb_per_split[i] = P.k_blocks[i];
     P.n_tiles[i] = (f.N + BN_OUT - 1) / BN_OUT;
+    P.idesc[i] = umma_idesc_bf16(BM, MMA_N);
+    P.b_bytes[i] = B_BYTES;
   }
   P.nprob = np;
   P.limit = limit;
@@ -490,6 +558,44 @@ cudaError_t launch_impl(const FfnProblem* routed, const FfnProblem* shared, floa
 }
 
 }  // namespace
+
+cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
+                               int32_t* err, int num_sms, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  GemmParams P;
+  memset(&P, 0, sizeof(P));
+  const int n_mma = router_mma_n(E);
+  if (!encode_a(&P.tma_a[0], x, T, H)) return cudaErrorInvalidValue;
+  if (!encode_b(&P.tma_b[0], w_split, 3, E, H, n_mma)) return cudaErrorInvalidValue;
+  P.offsets[0] = nullptr;
+  P.out_f32 = part;
+  P.groups[0] = 1;
+  P.rows[0] = T;
+  P.n_out[0] = E;
+  P.k_blocks[0] = (H + BK - 1) / BK;
+  P.k_parts[0] = 3;
+  const int total = 3 * P.k_blocks[0];
+  const int kbps = (total + k_splits - 1) / k_splits;
+  P.kb_per_split[0] = kbps;
+  P.k_splits[0] = (total + kbps - 1) / kbps;
+  P.n_tiles[0] = ((E + n_mma - 1) / n_mma) * P.k_splits[0];
+  P.idesc[0] = umma_idesc_bf16(BM, n_mma);
+  P.b_bytes[0] = n_mma * BK * 2;
+  P.nprob = 1;
+  P.err = err;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(grouped_gemm_kernel<Mode::Router>),
+                                   static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int tiles = ((T + BM - 1) / BM) * P.n_tiles[0];
+  grouped_gemm_kernel<Mode::Router><<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+int router_actual_splits(int H, int k_splits) {
+  const int total = 3 * ((H + BK - 1) / BK);
+  const int kbps = (total + k_splits - 1) / k_splits;
+  return (total + kbps - 1) / kbps;
+}
 
 cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
                                int num_sms, cudaStream_t stream) {

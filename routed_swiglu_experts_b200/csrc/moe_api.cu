@@ -104,21 +104,30 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   const int sms = num_sms_current_device();
   const bool with_shared = x_shared != nullptr && Is > 0 && T > 0;
 
+  // few tokens: the shared expert streams its weights with the split-K
+  // kernels; otherwise it is one more problem of the tcgen05 launches
+  const bool shared_small = with_shared && dense_small_ok(T, H, Is);
+  const bool shared_tc = with_shared && !shared_small;
   FfnProblem s_gu{}, s_d{};
-  if (with_shared) {
+  if (shared_tc) {
     s_gu = FfnProblem{x_shared, T, nullptr, 1, w.shared_w_gate_up, Is, H, hs, nullptr};
     s_d = FfnProblem{hs, T, nullptr, 1, w.shared_w_down, H, Is, shared_out, nullptr};
   }
+  if (shared_small)
+    MOE_CUDA_TRY(launch_dense_small_ffn(x_shared, T, H, Is, w.shared_w_gate_up, w.shared_w_down, cfg.swiglu_limit,
+                                        at<float>(ws, L.small_part), hs, shared_out, stream));
   if (!is_int4(cfg)) {
     FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
-    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, with_shared ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_gemm_down(&r_d, with_shared ? &s_d : nullptr, err, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, sms, stream));
   } else {
-    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, h, stream));
-    if (with_shared) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, w_perm, y_perm, stream));
-    if (with_shared) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
+    void* act16 = at<void>(ws, L.act16);
+    float* corr = at<float>(ws, L.act_corr);
+    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, corr, h, stream));
+    if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, R, act16, corr, w_perm, y_perm, stream));
+    if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
   }
   return MOE_OK;
 }
@@ -155,6 +164,7 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   };
   L.header = take(sizeof(WsHeader));
   L.logits = take(router_partial_floats(static_cast<int>(T), static_cast<int>(E)) * sizeof(float));
+  L.w_split = take(3 * E * H * 2);
   L.ids = take(R * sizeof(int32_t));
   L.wts = take(R * sizeof(float));
   L.offsets = take((E + 1) * sizeof(int32_t));
@@ -168,6 +178,11 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
   L.shared_out = take(T * H * 2);
+  const size_t kmax = std::max(H, I);
+  const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
+  L.act16 = take(int4 ? R * kmax * 2 : 0);
+  L.act_corr = take(int4 ? R * (kmax / 128) * sizeof(float) : 0);
+  L.small_part = take(Is > 0 ? dense_small_part_floats(static_cast<int>(H), static_cast<int>(Is)) * sizeof(float) : 0);
   L.total = off;
   return L;
 }
@@ -237,7 +252,8 @@ moe_status moe_router_topk(const moe_config* cfg, const moe_weights* w, const vo
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
-  return from_cuda(launch_router(*cfg, *w, x, T, topk_ids, topk_w, at<float>(ws, L.logits), stream));
+  return from_cuda(launch_router(*cfg, *w, x, T, topk_ids, topk_w, at<float>(ws, L.logits), at<void>(ws, L.w_split),
+                                 err_word(ws), num_sms_current_device(), stream));
 }
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const float* topk_w, const void* x, int32_t T,
@@ -303,7 +319,8 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   const WsLayout L = ws_layout(*cfg, T);
   int32_t* ids = topk_ids_opt != nullptr ? topk_ids_opt : at<int32_t>(ws, L.ids);
   float* wts = topk_w_opt != nullptr ? topk_w_opt : at<float>(ws, L.wts);
-  MOE_CUDA_TRY(launch_router(*cfg, *w, x, T, ids, wts, at<float>(ws, L.logits), stream));
+  MOE_CUDA_TRY(launch_router(*cfg, *w, x, T, ids, wts, at<float>(ws, L.logits), at<void>(ws, L.w_split),
+                             err_word(ws), num_sms_current_device(), stream));
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* row_of = at<int32_t>(ws, L.row_of);
   float* w_perm = at<float>(ws, L.w_perm);

@@ -13,22 +13,28 @@ namespace moe {
 // (cached per device and kernel).
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 
-// Router: rows of fp32 partial logits the split-H pass may use (per expert).
-constexpr int kRouterPartialRows = 8192;
-// Near-tie width on the fp32 biased score (2^-15) below which a token's
-// selection is re-ranked from fp64 logits.
-constexpr float kRouterTieTau = 3.0517578125e-05f;
+// Router: rows of fp32 partial logits (k-splits x tokens) the logits GEMM
+// may write, per expert.
+constexpr int kRouterPartialRows = 32768;
+// Near-tie width on the fp32 biased score (2^-13) below which adjacent
+// experts are re-ordered from fp64 logits.  It is far above the error of the
+// tensor-core fp32 logits (exact bf16 x bf16 products, fp32 sums over K).
+constexpr float kRouterTieTau = 1.220703125e-04f;
+
+// MMA N of the router GEMM: E rounded up to 16, at most 256.
+inline int router_mma_n(int E) { return std::min(256, (E + 15) / 16 * 16); }
 
 struct RouterPlan {
-  int bt;           // tokens per block
-  int ks;           // splits of H
-  int k_per_split;  // H elements per split (multiple of 32)
+  int ks;  // k-splits of the logits GEMM (partials summed by the top-k kernel)
 };
 RouterPlan router_plan(int T, int E, int H);
 size_t router_partial_floats(int Tmax, int E);
 size_t router_topk_smem(int E);
+int router_actual_splits(int H, int k_splits);
+cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
+                               int32_t* err, int num_sms, cudaStream_t stream);
 cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const void* x, int T, int32_t* ids,
-                          float* wts, float* part, cudaStream_t stream);
+                          float* wts, float* part, void* w_split, int32_t* err, int num_sms, cudaStream_t stream);
 
 // Permute: slots per counting block.
 constexpr int kPermChunk = 2048;
@@ -60,15 +66,26 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
                              cudaStream_t stream);
 
 // W4A16 routed expert kernels (dequantise in registers).
+// act16 / corr: scratch for the activations in MMA slot order (fp16,
+// [rows, K]) and their per-128-group corrections (fp32, [rows, K/128]).
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, void* h, cudaStream_t stream);
+                                const int32_t* offsets, int rows, void* act16, float* corr, void* h,
+                                cudaStream_t stream);
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const void* h, const int32_t* offsets,
-                              const float* w_perm, void* y_perm, cudaStream_t stream);
+                              int rows, void* act16, float* corr, const float* w_perm, void* y_perm,
+                              cudaStream_t stream);
+
+// Shared expert for T <= 32 tokens: split-K weight-streaming kernels.
+constexpr int kDenseSmallMaxSplits = 8;
+bool dense_small_ok(int T, int H, int Is);
+size_t dense_small_part_floats(int H, int Is);
+cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const void* w_gu, const void* w_d, float L,
+                                   float* part, void* h_s, void* out, cudaStream_t stream);
 
 // Workspace layout (byte offsets from the workspace base; 256-aligned).
 struct WsLayout {
-  size_t header, logits, ids, wts, offsets, row_of, src, w_perm, block_base, local_rank;
-  size_t x_perm, h, h_shared, y_perm, shared_out, total;
+  size_t header, logits, w_split, ids, wts, offsets, row_of, src, w_perm, block_base, local_rank;
+  size_t x_perm, h, h_shared, y_perm, shared_out, act16, act_corr, small_part, total;
 };
 WsLayout ws_layout(const moe_config& cfg, int Tmax);
 

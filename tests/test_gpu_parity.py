@@ -46,6 +46,9 @@ EDGE = {
     "w4a16_small": LayerConfig("w4a16_small", T=20, H=256, E=6, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
                                bias_range=0.05, w4a16=True),
     "w4a16_many_tokens": LayerConfig("w4a16_many_tokens", T=96, H=384, E=3, k=2, I=256, I_s=0, w4a16=True),
+    "shared_small_t32": LayerConfig("shared_small_t32", T=32, H=256, E=4, k=2, I=64, I_s=96, alpha=2.5,
+                                    renorm=True),
+    "shared_tc_t33": LayerConfig("shared_tc_t33", T=33, H=256, E=4, k=2, I=64, I_s=96),
 }
 
 
