@@ -2,7 +2,7 @@
 // split-K kernel.  With so few tokens the shared expert is bound by reading
 // its bf16 weights once from HBM; a 128-row tcgen05 tile would leave most
 // SMs idle (only I_s/128 tiles), so here every warp streams 16 weight rows
-// over one K slice with 16-byte loads and uses mma.sync m16n8k16 (bf16 in,
+// over one K slice through a cp.async ring and uses mma.sync m16n8k16 (bf16 in,
 // fp32 accumulate) as the dot-product engine; a second kernel adds the K
 // slices in a fixed order (deterministic) and applies the SwiGLU clamp
 // ("Module glm5next_mlp" §Numerics; the shared expert is added unscaled).
@@ -22,14 +22,6 @@ namespace {
 constexpr int kDsWarps = 8;
 constexpr int kDsTok = 32;  // tokens per call (4 n8 tiles)
 
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -41,16 +33,25 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 
 __device__ __forceinline__ uint4 and4(uint4 v, uint32_t m) { return make_uint4(v.x & m, v.y & m, v.z & m, v.w & m); }
 
+// Per-thread cp.async ring (same scheme as the W4A16 kernels): each 32-wide
+// k step a thread copies its two weight words and its four token words into
+// its own slots, kDsStages - 1 steps ahead of the MMAs.
+constexpr int kDsStages = 4;
+constexpr int kDsSlots = 6;
+constexpr size_t kDsSmem = static_cast<size_t>(kDsWarps) * kDsStages * kDsSlots * 32 * sizeof(uint4);
+
 // part[s][tile][16][32]: K-slice s of tile `tile` (blockIdx.x * 8 + warp).
 __global__ void __launch_bounds__(kDsWarps * 32)
     dense_small_kernel(const __nv_bfloat16* __restrict__ w, int K, int tiles, int gate_up, int half_rows,
                        const __nv_bfloat16* __restrict__ act, int T, int kslice, float* __restrict__ part) {
+  extern __shared__ __align__(16) uint4 ds_ring[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = lane >> 2, t = lane & 3;
   const int tile = blockIdx.x * kDsWarps + warp;
   const int s = blockIdx.y;
   if (tile >= tiles) return;
   const int k0 = s * kslice, k1 = min(K, k0 + kslice);
+  const int steps = (k1 - k0) / 32;
   // weight rows of tile rows g and g+8
   int ra, rb;
   if (gate_up) {
@@ -60,34 +61,48 @@ __global__ void __launch_bounds__(kDsWarps * 32)
     ra = tile * 16 + g;
     rb = ra + 8;
   }
-  const __nv_bfloat16* pa = w + static_cast<size_t>(ra) * K + 8 * t;
-  const __nv_bfloat16* pb = w + static_cast<size_t>(rb) * K + 8 * t;
+  const __nv_bfloat16* pa = w + static_cast<size_t>(ra) * K + k0 + 8 * t;
+  const __nv_bfloat16* pb = w + static_cast<size_t>(rb) * K + k0 + 8 * t;
   const __nv_bfloat16* px[4];
   uint32_t keep[4];
 #pragma unroll
   for (int n = 0; n < 4; ++n) {
     const int tok = g + 8 * n;
     keep[n] = tok < T ? 0xffffffffu : 0u;
-    px[n] = act + static_cast<size_t>(tok < T ? tok : 0) * K + 8 * t;
+    px[n] = act + static_cast<size_t>(tok < T ? tok : 0) * K + k0 + 8 * t;
   }
+  uint4* ring = ds_ring + static_cast<size_t>(warp) * kDsStages * kDsSlots * 32 + lane;
+  auto issue = [&](int i) {
+    uint4* st = ring + (i % kDsStages) * kDsSlots * 32;
+    cp_async16(st, pa + 32 * i);
+    cp_async16(st + 32, pb + 32 * i);
+#pragma unroll
+    for (int n = 0; n < 4; ++n) cp_async16(st + (2 + n) * 32, px[n] + 32 * i);
+  };
   float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
-#pragma unroll 4
-  for (int k = k0; k < k1; k += 32) {
-    const uint4 a = ld_stream16(pa + k);
-    const uint4 b = ld_stream16(pb + k);
-    uint4 xv[4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n) xv[n] = and4(__ldg(reinterpret_cast<const uint4*>(px[n] + k)), keep[n]);
+  for (int i = 0; i < kDsStages - 1; ++i) {
+    if (i < steps) issue(i);
+    cp_async_commit();
+  }
+  for (int i = 0; i < steps; ++i) {
+    cp_async_wait<kDsStages - 2>();
+    if (i + kDsStages - 1 < steps) issue(i + kDsStages - 1);
+    cp_async_commit();
+    const uint4* st = ring + (i % kDsStages) * kDsSlots * 32;
+    const uint4 a = st[0], b = st[32];
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
-      mma_bf16_16816(acc[n], a.x, b.x, a.y, b.y, xv[n].x, xv[n].y);
-      mma_bf16_16816(acc[n], a.z, b.z, a.w, b.w, xv[n].z, xv[n].w);
+      const uint4 xv = and4(st[(2 + n) * 32], keep[n]);
+      mma_bf16_16816(acc[n], a.x, b.x, a.y, b.y, xv.x, xv.y);
+      mma_bf16_16816(acc[n], a.z, b.z, a.w, b.w, xv.z, xv.w);
     }
   }
+  cp_async_wait<0>();
   // C fragment: acc[n][0..1] row g, tokens 8n + 2t, +1; acc[n][2..3] row g+8
   float* out = part + (static_cast<size_t>(s) * tiles + tile) * 16 * kDsTok;
 #pragma unroll
@@ -155,7 +170,9 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
   int S = splits_for(t_gu, H);
   int kslice = ((H + S - 1) / S + 31) / 32 * 32;
   S = (H + kslice - 1) / kslice;
-  dense_small_kernel<<<dim3((t_gu + kDsWarps - 1) / kDsWarps, S), kDsWarps * 32, 0, stream>>>(
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(dense_small_kernel), static_cast<int>(kDsSmem));
+  if (e != cudaSuccess) return e;
+  dense_small_kernel<<<dim3((t_gu + kDsWarps - 1) / kDsWarps, S), kDsWarps * 32, kDsSmem, stream>>>(
       static_cast<const __nv_bfloat16*>(w_gu), H, t_gu, 1, Is, static_cast<const __nv_bfloat16*>(x), T, kslice,
       part);
   dense_small_finish_kernel<<<(T * Is + 255) / 256, 256, 0, stream>>>(part, S, t_gu, 1, Is, T, L,
@@ -165,7 +182,7 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
   S = splits_for(t_d, Is);
   kslice = ((Is + S - 1) / S + 31) / 32 * 32;
   S = (Is + kslice - 1) / kslice;
-  dense_small_kernel<<<dim3((t_d + kDsWarps - 1) / kDsWarps, S), kDsWarps * 32, 0, stream>>>(
+  dense_small_kernel<<<dim3((t_d + kDsWarps - 1) / kDsWarps, S), kDsWarps * 32, kDsSmem, stream>>>(
       static_cast<const __nv_bfloat16*>(w_d), Is, t_d, 0, 0, static_cast<const __nv_bfloat16*>(h_s), T, kslice,
       part);
   dense_small_finish_kernel<<<(T * H + 255) / 256, 256, 0, stream>>>(part, S, t_d, 0, H, T, 0.f,

@@ -123,10 +123,9 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
     MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, sms, stream));
   } else {
     void* act16 = at<void>(ws, L.act16);
-    float* corr = at<float>(ws, L.act_corr);
-    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, corr, h, stream));
+    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, h, err, sms, stream));
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, R, act16, corr, w_perm, y_perm, stream));
+    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, R, act16, w_perm, y_perm, err, sms, stream));
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
   }
   return MOE_OK;
@@ -181,7 +180,6 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   const size_t kmax = std::max(H, I);
   const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
   L.act16 = take(int4 ? R * kmax * 2 : 0);
-  L.act_corr = take(int4 ? R * (kmax / 128) * sizeof(float) : 0);
   L.small_part = take(Is > 0 ? dense_small_part_floats(static_cast<int>(H), static_cast<int>(Is)) * sizeof(float) : 0);
   L.total = off;
   return L;

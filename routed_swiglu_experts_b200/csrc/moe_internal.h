@@ -13,6 +13,10 @@ namespace moe {
 // (cached per device and kernel).
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 
+// Encode a tiled TMA descriptor (strides in bytes for dims 1..rank-1).
+bool encode_tma(CUtensorMap* m, CUtensorMapDataType dtype, int rank, const void* base, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle);
+
 // Router: rows of fp32 partial logits (k-splits x tokens) the logits GEMM
 // may write, per expert.
 constexpr int kRouterPartialRows = 32768;
@@ -66,13 +70,12 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
                              cudaStream_t stream);
 
 // W4A16 routed expert kernels (dequantise in registers).
-// act16 / corr: scratch for the activations in MMA slot order (fp16,
-// [rows, K]) and their per-128-group corrections (fp32, [rows, K/128]).
+// act16: scratch for the activations in MMA slot order (fp16, [rows, K]).
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* corr, void* h,
+                                const int32_t* offsets, int rows, void* act16, void* h, int32_t* err, int num_sms,
                                 cudaStream_t stream);
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const void* h, const int32_t* offsets,
-                              int rows, void* act16, float* corr, const float* w_perm, void* y_perm,
+                              int rows, void* act16, const float* w_perm, void* y_perm, int32_t* err, int num_sms,
                               cudaStream_t stream);
 
 // Shared expert for T <= 32 tokens: split-K weight-streaming kernels.
@@ -85,7 +88,7 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
 // Workspace layout (byte offsets from the workspace base; 256-aligned).
 struct WsLayout {
   size_t header, logits, w_split, ids, wts, offsets, row_of, src, w_perm, block_base, local_rank;
-  size_t x_perm, h, h_shared, y_perm, shared_out, act16, act_corr, small_part, total;
+  size_t x_perm, h, h_shared, y_perm, shared_out, act16, small_part, total;
 };
 WsLayout ws_layout(const moe_config& cfg, int Tmax);
 
