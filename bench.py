@@ -185,14 +185,16 @@ def w4a16_bytes(cfg, ids):
 
 
 def launches_per_step(cfg):
-    """Kernels one forward launches (router 2, permute 3, combine 1, plus the
-    expert FFN path)."""
-    n = 6
+    """Kernels one forward launches: router 3 (weight split, tensor-core
+    logits, top-k), permute 3 (count/rank, scan, scatter), combine 1, plus the
+    expert FFN path."""
+    n = 7
     small_shared = cfg.I_s > 0 and cfg.T <= 32 and cfg.H % 32 == 0 and cfg.I_s % 32 == 0
+    shared = (4 if small_shared else 2) if cfg.I_s > 0 else 0
     if cfg.w4a16:
-        n += 4 + (4 if small_shared else (2 if cfg.I_s > 0 else 0))
+        n += 4 + shared          # routed: (prep + gemv) x 2
     else:
-        n += 2 + (4 if small_shared else 0)
+        n += 2 + (4 if small_shared else 0)  # routed + large shared share two launches
     return n
 
 

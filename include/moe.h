@@ -129,9 +129,11 @@ MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t st
 /* Router: logit[t, e] = sum_h x[t, h] * router_w[e, h] in fp32 ([beam]
  * beam_router_gating_linear; no linear bias); s = sigmoid(logit); the k
  * experts with the largest s + correction_bias, ties to the lower id
- * ([glm5next] §Numerics: the bias steers selection only).  Selections whose
- * fp32 biased scores are within 2^-15 of a neighbour are re-ranked from
- * fp64 logits so the ids equal the exact-arithmetic selection.
+ * ([glm5next] §Numerics: the bias steers selection only).  The logits run
+ * on the tensor cores with the fp32 weight split exactly into three bf16
+ * parts; selections whose fp32 biased scores are within 2^-13 of a neighbour
+ * are re-ranked from fp64 logits so the ids equal the exact-arithmetic
+ * selection.
  *   x         bf16 [T, H]
  *   topk_ids  int32 [T, k] out: selection order (biased desc, id asc)
  *   topk_w    fp32  [T, k] out: alpha * s_e (renormalised first if enabled),

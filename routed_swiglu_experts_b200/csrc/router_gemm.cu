@@ -1,0 +1,343 @@
+// Router logits on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// fp32 partial logits of x Wr^T with the fp32 router weight split exactly
+// into three bf16 parts (hi + mid + lo) that are concatenated along K, so
+// every bf16 x bf16 product is exact and the tensor core accumulates in fp32
+// ("bridge.models.beam.modeling_beam" beam_router_gating_linear: fp32
+// operands).  For small token counts the (parts x k-blocks) range is split
+// across CTAs; the top-k kernel sums the partials in a fixed order.
+//
+// Tile: 128 token rows x N = router_mma_n(E) columns, K step 64 (one
+// 128-byte swizzle atom).  Warps 0-3: epilogue (TMEM -> registers ->
+// global fp32), warp 4: TMA producer, warp 5: TMEM owner + MMA issuer.  A
+// 4-stage smem ring feeds the MMA; two TMEM accumulators let the epilogue of
+// tile i overlap the MMAs of tile i+1.  Every mbarrier wait is bounded; on
+// timeout the kernel records MOE_ERR_DEVICE_TIMEOUT in the workspace error
+// word, drains its own in-flight copies and MMAs, frees TMEM and returns.
+
+#include <cstring>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int MMA_N = 256;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int B_BYTES = MMA_N * BK * 2;    // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+struct alignas(64) RouterParams {
+  CUtensorMap tma_a;          // x: {H, T} box {64, 128}
+  CUtensorMap tma_b;          // split weight: {H, E, 3} box {64, n_mma, 1}
+  float* out_f32;             // partial logits [k_splits, rows, n_out]
+  int32_t rows;
+  int32_t n_out;
+  int32_t n_mma;              // MMA N (columns of one tile)
+  int32_t k_blocks;           // k-blocks of one pass over K
+  int32_t k_splits;           // tiles split along the (3 parts x k-blocks) range
+  int32_t kb_per_split;
+  int32_t n_tiles;            // output-column tiles x k_splits
+  uint32_t idesc;             // MMA instruction descriptor
+  int32_t* err;
+};
+
+struct SmemCtl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemCtl);
+static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory");
+
+struct TileInfo {
+  int row0;     // first token row of the tile
+  int nrows;    // valid rows (<= BM)
+  int nidx;     // output-column tile index
+  int split;    // k-split index
+};
+
+// Tile order: output-column tile (and k-split) major, row tile minor.
+__device__ __forceinline__ TileInfo decode_tile(const RouterParams& P, int t) {
+  TileInfo ti;
+  const int mtiles = (P.rows + BM - 1) / BM;
+  int nidx = t / mtiles;
+  const int m = t - nidx * mtiles;
+  ti.row0 = m * BM;
+  ti.nrows = min(BM, P.rows - ti.row0);
+  ti.split = nidx % P.k_splits;
+  ti.nidx = nidx / P.k_splits;
+  return ti;
+}
+
+// k-blocks [kb0, kb1) of the (parts x k-blocks) range a tile accumulates.
+__device__ __forceinline__ void tile_k_range(const RouterParams& P, const TileInfo& ti, int& kb0, int& kb1) {
+  const int total = P.k_blocks * 3;
+  kb0 = ti.split * P.kb_per_split;
+  kb1 = min(total, kb0 + P.kb_per_split);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) router_gemm_kernel(const __grid_constant__ RouterParams P) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  unsigned char* smem_a = smem;
+  unsigned char* smem_b = smem + STAGES * A_BYTES;
+  SmemCtl& c = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&c.tmem_full[a], 1);
+      mbar_init(&c.tmem_empty[a], 4 * 32);
+    }
+    mbar_init(&c.mma_done, 1);
+    c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&P.tma_a);
+    tma_prefetch_desc(&P.tma_b);
+  }
+  if (warp == 5) tmem_alloc(&c.tmem_base, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = c.tmem_base;
+  const int total_tiles = ((P.rows + BM - 1) / BM) * P.n_tiles;
+  volatile int32_t* abort_flag = &c.abort_flag;
+
+  auto fail = [&](int detail) {
+    *abort_flag = 1;
+    report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, detail);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(P, t);
+        const int ncol0 = ti.nidx * P.n_mma;
+        int kb0, kb1;
+        tile_k_range(P, ti, kb0, kb1);
+        const uint32_t stage_tx = static_cast<uint32_t>(A_BYTES + P.n_mma * BK * 2);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+            fail(1);
+            ok = false;
+            break;
+          }
+          const int part = kb / P.k_blocks;
+          const int kc = (kb - part * P.k_blocks) * BK;
+          mbar_arrive_expect_tx(&c.full[stage], stage_tx);
+          tma_load_2d(smem_a + stage * A_BYTES, &P.tma_a, kc, ti.row0, &c.full[stage]);
+          tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b, kc, ncol0, part, &c.full[stage]);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // drain: wait (bounded) for the last copy issued to each stage
+      const int nst = issued < STAGES ? issued : STAGES;
+      for (int j = 0; j < nst; ++j) {
+        const int i = issued - 1 - j;
+        const int s = i % STAGES;
+        const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
+        volatile int32_t never = 0;
+        if (!mbar_wait_bounded(&c.full[s], par, &never, kTimeoutNs)) report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, 9);
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile(P, t);
+        const uint32_t idesc = P.idesc;
+        int kb0, kb1;
+        tile_k_range(P, ti, kb0, kb1);
+        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          fail(2);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
+            fail(3);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem_a + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(smem_b + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
+            const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&c.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&c.tmem_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // drain every MMA this thread issued before TMEM is released
+      umma_commit(&c.mma_done);
+      volatile int32_t never = 0;
+      if (!mbar_wait_bounded(&c.mma_done, 0, &never, kTimeoutNs)) report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, 8);
+    }
+  } else {
+    // ------------------------------------------- epilogue (warps 0 .. 3) --
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const int row_in_tile = warp * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const TileInfo ti = decode_tile(P, t);
+      const int ncol0 = ti.nidx * P.n_mma;
+      // every lane waits; the outcome is made warp-uniform before the
+      // warp-collective TMEM loads
+      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) fail(4);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * MMA_N);
+      const bool row_ok = row_in_tile < ti.nrows;
+      const int N = P.n_out;
+      const int nch = (P.n_mma + 31) / 32;
+      float* frow = P.out_f32 + (static_cast<size_t>(ti.split) * P.rows + ti.row0 + (row_ok ? row_in_tile : 0)) * N;
+#pragma unroll 1
+      for (int ch = 0; ch < nch; ++ch) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tbase + ch * 32, v);
+        tmem_ld_wait();
+        if (ch == nch - 1) {
+          tc_fence_before();
+          mbar_arrive(&c.tmem_empty[acc]);
+        }
+        const int col = ncol0 + ch * 32;
+        if (row_ok) {
+          if ((N & 3) == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (col + 4 * q < N)
+                *reinterpret_cast<uint4*>(frow + col + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                                                           v[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (col + q < N) frow[col + q] = __uint_as_float(v[q]);
+          }
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host --
+
+// 2-D bf16 map over [rows, K] (K innermost), box 64 x 128, 128-byte swizzle.
+bool encode_a(CUtensorMap* m, const void* base, int rows, int K) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {BK, BM};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// 3-D bf16 map over [slices, N, K] (K innermost), box 64 x box_n x 1.
+bool encode_b(CUtensorMap* m, const void* base, int slices, int N, int K, int box_n) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), static_cast<uint64_t>(slices)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * N * 2};
+  const uint32_t box[3] = {BK, static_cast<uint32_t>(box_n), 1};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
+                               int32_t* err, int num_sms, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  RouterParams P;
+  memset(&P, 0, sizeof(P));
+  const int n_mma = router_mma_n(E);
+  if (!encode_a(&P.tma_a, x, T, H)) return cudaErrorInvalidValue;
+  if (!encode_b(&P.tma_b, w_split, 3, E, H, n_mma)) return cudaErrorInvalidValue;
+  P.out_f32 = part;
+  P.rows = T;
+  P.n_out = E;
+  P.n_mma = n_mma;
+  P.k_blocks = (H + BK - 1) / BK;
+  const int total = 3 * P.k_blocks;
+  const int kbps = (total + k_splits - 1) / k_splits;
+  P.kb_per_split = kbps;
+  P.k_splits = (total + kbps - 1) / kbps;
+  P.n_tiles = ((E + n_mma - 1) / n_mma) * P.k_splits;
+  P.idesc = umma_idesc_bf16(BM, n_mma);
+  P.err = err;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(router_gemm_kernel), static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int tiles = ((T + BM - 1) / BM) * P.n_tiles;
+  router_gemm_kernel<<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+int router_actual_splits(int H, int k_splits) {
+  const int total = 3 * ((H + BK - 1) / BK);
+  const int kbps = (total + k_splits - 1) / k_splits;
+  return (total + kbps - 1) / kbps;
+}
+
+}  // namespace moe
