@@ -115,17 +115,20 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   }
   if (shared_small)
     MOE_CUDA_TRY(launch_dense_small_ffn(x_shared, T, H, Is, w.shared_w_gate_up, w.shared_w_down, cfg.swiglu_limit,
-                                        at<float>(ws, L.small_part), hs, shared_out, stream));
+                                        at<float>(ws, L.small_part), hs, shared_out, err, sms, stream));
   if (!is_int4(cfg)) {
     FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
     MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
     MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, sms, stream));
   } else {
+    // gate/up in fp32 into the h region; the SwiGLU is applied while the
+    // down projection's activations are prepared
     void* act16 = at<void>(ws, L.act16);
-    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, h, err, sms, stream));
+    float* gu = at<float>(ws, L.h);
+    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, stream));
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, h, offsets, R, act16, w_perm, y_perm, err, sms, stream));
+    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, stream));
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
   }
   return MOE_OK;
@@ -173,12 +176,12 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.block_base = take(static_cast<size_t>(perm_blocks(static_cast<int>(R))) * E * sizeof(int32_t));
   L.local_rank = take(R * sizeof(int32_t));
   L.x_perm = take(R * H * 2);
-  L.h = take(R * I * 2);
+  const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
+  L.h = take(int4 ? R * 2 * I * 4 : R * I * 2);  // int4: fp32 gate/up; bf16: h
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
   L.shared_out = take(T * H * 2);
   const size_t kmax = std::max(H, I);
-  const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
   L.act16 = take(int4 ? R * kmax * 2 : 0);
   L.small_part = take(Is > 0 ? dense_small_part_floats(static_cast<int>(H), static_cast<int>(Is)) * sizeof(float) : 0);
   L.total = off;

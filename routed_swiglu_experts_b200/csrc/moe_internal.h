@@ -34,6 +34,11 @@ struct RouterPlan {
 RouterPlan router_plan(int T, int E, int H);
 size_t router_partial_floats(int Tmax, int E);
 size_t router_topk_smem(int E);
+// Split-K tensor-core GEMM with fp32 partials part[s][rows][N] over `parts`
+// passes of K (B slice p per pass); n_mma: MMA N, a multiple of 16 <= 256.
+cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, int parts, int N, int n_mma,
+                               int k_splits, float* part, int32_t* err, int num_sms, cudaStream_t stream);
+int splitk_actual_splits(int K, int parts, int k_splits);
 int router_actual_splits(int H, int k_splits);
 cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
                                int32_t* err, int num_sms, cudaStream_t stream);
@@ -72,18 +77,18 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
 // W4A16 routed expert kernels (dequantise in registers).
 // act16: scratch for the activations in MMA slot order (fp16, [rows, K]).
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, void* h, int32_t* err, int num_sms,
-                                cudaStream_t stream);
-cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const void* h, const int32_t* offsets,
-                              int rows, void* act16, const float* w_perm, void* y_perm, int32_t* err, int num_sms,
-                              cudaStream_t stream);
+                                const int32_t* offsets, int rows, void* act16, float* gu, cudaStream_t stream);
+cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
+                              int rows, void* act16, const float* w_perm, void* y_perm, cudaStream_t stream);
 
-// Shared expert for T <= 32 tokens: split-K weight-streaming kernels.
-constexpr int kDenseSmallMaxSplits = 8;
+// Shared expert for T <= 32 tokens: split-K tensor-core GEMMs streaming the
+// weights across all SMs, then an ordered sum of the K slices.
+constexpr int kDenseSmallMaxTokens = 32;
+constexpr int kDenseSmallMaxSplits = 16;
 bool dense_small_ok(int T, int H, int Is);
 size_t dense_small_part_floats(int H, int Is);
 cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const void* w_gu, const void* w_d, float L,
-                                   float* part, void* h_s, void* out, cudaStream_t stream);
+                                   float* part, void* h_s, void* out, int32_t* err, int num_sms, cudaStream_t stream);
 
 // Workspace layout (byte offsets from the workspace base; 256-aligned).
 struct WsLayout {

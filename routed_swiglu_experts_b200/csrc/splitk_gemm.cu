@@ -1,20 +1,25 @@
-// Router logits on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// Split-K GEMM with fp32 partial outputs on the sm_100a tensor cores
+// (tcgen05 + TMEM + TMA):  part[s][r][n] = sum over K-slice s of
+// A[r, k] * B[p, n, k], where the K range is `parts` passes over the
+// reduction length, pass p reading slice p of B.  Two users:
+//  * router logits: the fp32 router weight split exactly into three bf16
+//    parts (hi + mid + lo), so every bf16 x bf16 product is exact and the
+//    tensor core accumulates in fp32 ("bridge.models.beam.modeling_beam"
+//    beam_router_gating_linear: fp32 operands); parts = 3;
+//  * the shared expert for a handful of tokens ("Module glm5next_mlp",
+//    FFN_MODULE: the dense SwiGLU FFN also serves the shared expert): with so
+//    few rows the projection is bound by streaming its bf16 weight once, so
+//    K is split until every SM streams a slice; parts = 1.
+// The caller sums the K slices in a fixed order (deterministic).
 //
-// fp32 partial logits of x Wr^T with the fp32 router weight split exactly
-// into three bf16 parts (hi + mid + lo) that are concatenated along K, so
-// every bf16 x bf16 product is exact and the tensor core accumulates in fp32
-// ("bridge.models.beam.modeling_beam" beam_router_gating_linear: fp32
-// operands).  For small token counts the (parts x k-blocks) range is split
-// across CTAs; the top-k kernel sums the partials in a fixed order.
-//
-// Tile: 128 token rows x N = router_mma_n(E) columns, K step 64 (one
-// 128-byte swizzle atom).  Warps 0-3: epilogue (TMEM -> registers ->
-// global fp32), warp 4: TMA producer, warp 5: TMEM owner + MMA issuer.  A
-// 4-stage smem ring feeds the MMA; two TMEM accumulators let the epilogue of
-// tile i overlap the MMAs of tile i+1.  Every mbarrier wait is bounded; on
-// timeout the kernel records MOE_ERR_DEVICE_TIMEOUT in the workspace error
-// word, drains its own in-flight copies and MMAs, frees TMEM and returns.
-
+// Tile: 128 A rows x n_mma (<= 256) columns, K step 64 (one 128-byte
+// swizzle atom); rows past the end of A are zero-filled by TMA and never
+// stored.  Warps 0-3: epilogue (TMEM -> registers -> global fp32), warp 4:
+// TMA producer, warp 5: TMEM owner + MMA issuer.  A 4-stage smem ring feeds
+// the MMA; two TMEM accumulators let the epilogue of tile i overlap the MMAs
+// of tile i+1.  Every mbarrier wait is bounded; on timeout the kernel records
+// MOE_ERR_DEVICE_TIMEOUT in the workspace error word, drains its own
+// in-flight copies and MMAs, frees TMEM and returns.
 #include <cstring>
 
 #include "moe_internal.h"
@@ -34,15 +39,16 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 
-struct alignas(64) RouterParams {
-  CUtensorMap tma_a;          // x: {H, T} box {64, 128}
-  CUtensorMap tma_b;          // split weight: {H, E, 3} box {64, n_mma, 1}
+struct alignas(64) SplitKParams {
+  CUtensorMap tma_a;          // A: {K, rows} box {64, 128}
+  CUtensorMap tma_b;          // B: {K, N, parts} box {64, n_mma, 1}
   float* out_f32;             // partial logits [k_splits, rows, n_out]
   int32_t rows;
   int32_t n_out;
   int32_t n_mma;              // MMA N (columns of one tile)
   int32_t k_blocks;           // k-blocks of one pass over K
-  int32_t k_splits;           // tiles split along the (3 parts x k-blocks) range
+  int32_t parts;              // passes over K (slices of B)
+  int32_t k_splits;           // tiles split along the (parts x k-blocks) range
   int32_t kb_per_split;
   int32_t n_tiles;            // output-column tiles x k_splits
   uint32_t idesc;             // MMA instruction descriptor
@@ -70,7 +76,7 @@ struct TileInfo {
 };
 
 // Tile order: output-column tile (and k-split) major, row tile minor.
-__device__ __forceinline__ TileInfo decode_tile(const RouterParams& P, int t) {
+__device__ __forceinline__ TileInfo decode_tile(const SplitKParams& P, int t) {
   TileInfo ti;
   const int mtiles = (P.rows + BM - 1) / BM;
   int nidx = t / mtiles;
@@ -83,13 +89,13 @@ __device__ __forceinline__ TileInfo decode_tile(const RouterParams& P, int t) {
 }
 
 // k-blocks [kb0, kb1) of the (parts x k-blocks) range a tile accumulates.
-__device__ __forceinline__ void tile_k_range(const RouterParams& P, const TileInfo& ti, int& kb0, int& kb1) {
-  const int total = P.k_blocks * 3;
+__device__ __forceinline__ void tile_k_range(const SplitKParams& P, const TileInfo& ti, int& kb0, int& kb1) {
+  const int total = P.k_blocks * P.parts;
   kb0 = ti.split * P.kb_per_split;
   kb1 = min(total, kb0 + P.kb_per_split);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) router_gemm_kernel(const __grid_constant__ RouterParams P) {
+__global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_constant__ SplitKParams P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -307,37 +313,45 @@ bool encode_b(CUtensorMap* m, const void* base, int slices, int N, int K, int bo
 
 }  // namespace
 
-cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
-                               int32_t* err, int num_sms, cudaStream_t stream) {
-  if (T <= 0) return cudaSuccess;
-  RouterParams P;
+cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, int parts, int N, int n_mma,
+                               int k_splits, float* part, int32_t* err, int num_sms, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  if (n_mma < 16 || n_mma > 256 || n_mma % 16 != 0 || parts < 1) return cudaErrorInvalidValue;
+  SplitKParams P;
   memset(&P, 0, sizeof(P));
-  const int n_mma = router_mma_n(E);
-  if (!encode_a(&P.tma_a, x, T, H)) return cudaErrorInvalidValue;
-  if (!encode_b(&P.tma_b, w_split, 3, E, H, n_mma)) return cudaErrorInvalidValue;
+  if (!encode_a(&P.tma_a, a, rows, K)) return cudaErrorInvalidValue;
+  if (!encode_b(&P.tma_b, b, parts, N, K, n_mma)) return cudaErrorInvalidValue;
   P.out_f32 = part;
-  P.rows = T;
-  P.n_out = E;
+  P.rows = rows;
+  P.n_out = N;
   P.n_mma = n_mma;
-  P.k_blocks = (H + BK - 1) / BK;
-  const int total = 3 * P.k_blocks;
+  P.k_blocks = (K + BK - 1) / BK;
+  P.parts = parts;
+  const int total = parts * P.k_blocks;
   const int kbps = (total + k_splits - 1) / k_splits;
   P.kb_per_split = kbps;
   P.k_splits = (total + kbps - 1) / kbps;
-  P.n_tiles = ((E + n_mma - 1) / n_mma) * P.k_splits;
+  P.n_tiles = ((N + n_mma - 1) / n_mma) * P.k_splits;
   P.idesc = umma_idesc_bf16(BM, n_mma);
   P.err = err;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(router_gemm_kernel), static_cast<int>(kSmemBytes));
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const int tiles = ((T + BM - 1) / BM) * P.n_tiles;
-  router_gemm_kernel<<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
+  const int tiles = ((rows + BM - 1) / BM) * P.n_tiles;
+  splitk_gemm_kernel<<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
-int router_actual_splits(int H, int k_splits) {
-  const int total = 3 * ((H + BK - 1) / BK);
+int splitk_actual_splits(int K, int parts, int k_splits) {
+  const int total = parts * ((K + BK - 1) / BK);
   const int kbps = (total + k_splits - 1) / k_splits;
   return (total + kbps - 1) / kbps;
 }
+
+cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
+                               int32_t* err, int num_sms, cudaStream_t stream) {
+  return launch_splitk_gemm(x, T, H, w_split, 3, E, router_mma_n(E), k_splits, part, err, num_sms, stream);
+}
+
+int router_actual_splits(int H, int k_splits) { return splitk_actual_splits(H, 3, k_splits); }
 
 }  // namespace moe

@@ -1,10 +1,10 @@
 // W4A16 routed expert projections for small token counts ("Module
 // glm5next_mlp", W4A16_GEMV_MODULE: its GEMV kernels run every routed-expert
 // projection except the grouped prefill GEMM).  HBM-bound: every weight byte
-// is read once per (expert, 8-token chunk) through a per-thread cp.async
-// ring, dequantised in registers and fed to mma.sync m16n8k16 (fp16 in,
-// fp32 accumulate) as a dot-product engine, which keeps the ALU work per 8
-// codes to one shift and four LOP3s.
+// is read once per (expert, 8-token chunk) with streaming 16-byte loads,
+// dequantised in registers and fed to mma.sync m16n8k16 (fp16 in, fp32
+// accumulate) as a dot-product engine, which keeps the ALU work per 8 codes
+// to one shift, four LOP3s and four fp16x2 subtractions.
 //
 // Weight format: uint8 [N, K/2], the code of k = 2c in the low nibble of byte
 // c and k = 2c+1 in the high nibble; w = (code - 8) * scale[n, k / 128].
@@ -87,8 +87,6 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
 
 __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-__device__ __forceinline__ uint4 and4(uint4 v, uint32_t m) { return make_uint4(v.x & m, v.y & m, v.z & m, v.w & m); }
-
 // Activations in MMA slot order.  One thread per 8 consecutive values of a
 // row: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16}.
 __global__ void __launch_bounds__(256)
@@ -108,21 +106,61 @@ __global__ void __launch_bounds__(256)
   act16[idx] = o;
 }
 
-// Streaming GEMV.  One warp owns 16 output rows of each matrix (gate and up
-// for the gate/up kernel) for one expert and one 8-token chunk, and walks K
-// one 128-wide scale group at a time: per group each thread loads 16 code
-// bytes of rows g and g+8 of each matrix (64 contiguous bytes per row per
-// warp), its token's 64 activation bytes (only the lanes whose token exists
-// load), and every 8 groups one 16-byte word of 8 scales per row, prefetched
-// a batch ahead.  Many small blocks (4 warps) keep enough loads in flight.
-constexpr int kGemvWarps = 4;
-constexpr int kGemvRows = 16 * kGemvWarps;  // output rows per block per matrix
+// Down-projection activations: the clamped SwiGLU of the fp32 gate/up
+// projection ("Module glm5next_mlp" §Numerics), rounded to bf16 like the
+// bf16 path's h, then laid out in MMA slot order as above.  gu: fp32
+// [rows, 2I] (gate columns [0, I), up columns [I, 2I)); one thread per 8
+// consecutive features of a row.
+__global__ void __launch_bounds__(256)
+    w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n8) return;
+  const int i8 = I / 8;
+  const long long r = idx / i8;
+  const int f = static_cast<int>(idx - r * i8) * 8;
+  const float* gp = gu + r * 2 * I + f;
+  const float4 g0 = __ldg(reinterpret_cast<const float4*>(gp)), g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
+  const float4 u0 = __ldg(reinterpret_cast<const float4*>(gp + I)), u1 = __ldg(reinterpret_cast<const float4*>(gp + I + 4));
+  const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  float h[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float gc = fminf(gv[j], L);
+    const float uc = fminf(fmaxf(uv[j], -L), L);
+    h[j] = __bfloat162float(__float2bfloat16_rn(__fdividef(gc, 1.f + __expf(-gc)) * uc));
+  }
+  const __half2 a04 = __floats2half2_rn(h[0], h[4]);
+  const __half2 b15 = __floats2half2_rn(h[1] * 0.0625f, h[5] * 0.0625f);
+  const __half2 a26 = __floats2half2_rn(h[2], h[6]);
+  const __half2 b37 = __floats2half2_rn(h[3] * 0.0625f, h[7] * 0.0625f);
+  uint4 o;
+  o.x = *reinterpret_cast<const uint32_t*>(&a04);
+  o.y = *reinterpret_cast<const uint32_t*>(&b15);
+  o.z = *reinterpret_cast<const uint32_t*>(&a26);
+  o.w = *reinterpret_cast<const uint32_t*>(&b37);
+  act16[idx] = o;
+}
 
-template <int NM>
+// Streaming GEMV.  One warp owns 16 output rows of one expert for one
+// 8-token chunk and walks K one 128-wide scale group at a time: per group
+// each thread loads 16 code bytes of rows g and g+8 (64 contiguous bytes per
+// row per warp), its token's 64 activation bytes (only the lanes whose token
+// exists load), and every 8 groups one 16-byte word of 8 scales per row,
+// prefetched a batch ahead.  Many small blocks (4 warps, 70 registers) keep
+// enough loads in flight.  The gate/up projection runs as one matrix of 2I
+// rows with fp32 output (the SwiGLU is applied when the down projection's
+// activations are prepared); the down projection writes bf16 scaled by the
+// row's combine weight.
+constexpr int kGemvWarps = 4;
+constexpr int kGemvRows = 16 * kGemvWarps;  // output rows per block
+
+template <bool F32OUT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     w4a16_gemv_kernel(const uint4* __restrict__ act16, const int32_t* __restrict__ offsets,
                       const uint8_t* __restrict__ q, const __nv_bfloat16* __restrict__ scales, int N, int K,
-                      float limit, const float* __restrict__ w_perm, __nv_bfloat16* __restrict__ out) {
+                      const float* __restrict__ w_perm, void* __restrict__ out) {
+  constexpr int NM = 1;
   const int e = blockIdx.y;
   const int r_begin = offsets[e], r_end = offsets[e + 1];
   if (r_end <= r_begin) return;
@@ -216,15 +254,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
       const int col = n0 + g + 8 * (cc >> 1);
       if (tok < ntok) {
         const int r = tc + tok;
-        float v;
-        if (NM == 2) {
-          const float gv = fminf(acc[0][cc], limit);
-          const float uv = fminf(fmaxf(acc[NM - 1][cc], -limit), limit);
-          v = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+        if (F32OUT) {
+          static_cast<float*>(out)[static_cast<size_t>(r) * N + col] = acc[0][cc];
         } else {
-          v = acc[0][cc] * (w_perm != nullptr ? w_perm[r] : 1.f);
+          const float v = acc[0][cc] * (w_perm != nullptr ? w_perm[r] : 1.f);
+          static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(r) * N + col] = __float2bfloat16_rn(v);
         }
-        out[static_cast<size_t>(r) * N + col] = __float2bfloat16_rn(v);
       }
     }
   }
@@ -237,39 +272,38 @@ cudaError_t launch_prep(const void* act, int rows, int K, void* act16, cudaStrea
   return cudaGetLastError();
 }
 
-template <int NM>
+template <bool F32OUT>
 cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, const void* act16,
-                        const int32_t* offsets, const float* w_perm, float limit, void* out, cudaStream_t stream) {
+                        const int32_t* offsets, const float* w_perm, void* out, cudaStream_t stream) {
   const dim3 grid((N + kGemvRows - 1) / kGemvRows, E);
-  w4a16_gemv_kernel<NM><<<grid, kGemvWarps * 32, 0, stream>>>(
+  w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, 0, stream>>>(
       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
-      static_cast<const __nv_bfloat16*>(scales), N, K, limit, w_perm, static_cast<__nv_bfloat16*>(out));
+      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, void* h, int32_t* err, int num_sms,
-                                cudaStream_t stream) {
+                                const int32_t* offsets, int rows, void* act16, float* gu, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
   cudaError_t e = launch_prep(x_perm, rows, H, act16, stream);
   if (e != cudaSuccess) return e;
-  // W_gu [E, 2I, H/2] viewed as [2E, I, H/2]: slice 2e = gate, 2e+1 = up
-  (void)err;
-  (void)num_sms;
-  return launch_gemv<2>(w.w_gate_up, w.s_gate_up, E, I, H, act16, offsets, nullptr, cfg.swiglu_limit, h, stream);
+  // W_gu [E, 2I, H/2]: one matrix of 2I rows per expert (gate rows, then up rows)
+  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, stream);
 }
 
-cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const void* h, const int32_t* offsets,
-                              int rows, void* act16, const float* w_perm, void* y_perm, int32_t* err, int num_sms,
-                              cudaStream_t stream) {
+cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
+                              int rows, void* act16, const float* w_perm, void* y_perm, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
-  cudaError_t e = launch_prep(h, rows, I, act16, stream);
-  if (e != cudaSuccess) return e;
-  (void)err;
-  (void)num_sms;
-  return launch_gemv<1>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, 0.f, y_perm, stream);
+  const long long n8 = static_cast<long long>(rows) * (I / 8);
+  if (n8 > 0) {
+    w4a16_prep_swiglu_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+        gu, I, n8, cfg.swiglu_limit, static_cast<uint4*>(act16));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, stream);
 }
 
 }  // namespace moe
