@@ -1,7 +1,7 @@
 // W4A16 routed expert projections for small token counts ("Module
 // glm5next_mlp", W4A16_GEMV_MODULE: its GEMV kernels run every routed-expert
 // projection except the grouped prefill GEMM).  HBM-bound: every weight byte
-// is read once per (expert, 8-token chunk) with streaming 16-byte loads,
+// is read once per (expert, 8-token chunk) through a per-warp cp.async ring,
 // dequantised in registers and fed to mma.sync m16n8k16 (fp16 in, fp32
 // accumulate) as a dot-product engine, which keeps the ALU work per 8 codes
 // to one shift, four LOP3s and four fp16x2 subtractions.
@@ -35,12 +35,6 @@ namespace moe {
 namespace {
 
 constexpr int kTok = 8;  // tokens per work item (the MMA's N)
-
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                               uint32_t b0, uint32_t b1) {
@@ -143,24 +137,30 @@ __global__ void __launch_bounds__(256)
 }
 
 // Streaming GEMV.  One warp owns 16 output rows of one expert for one
-// 8-token chunk and walks K one 128-wide scale group at a time: per group
-// each thread loads 16 code bytes of rows g and g+8 (64 contiguous bytes per
-// row per warp), its token's 64 activation bytes (only the lanes whose token
-// exists load), and every 8 groups one 16-byte word of 8 scales per row,
-// prefetched a batch ahead.  Many small blocks (4 warps, 70 registers) keep
-// enough loads in flight.  The gate/up projection runs as one matrix of 2I
+// 8-token chunk and walks K one 128-wide scale group at a time.  The code
+// stream is the latency problem: each thread copies its 16 code bytes of rows
+// g and g+8 per group into its own slots of a per-warp shared-memory ring
+// with cp.async, kGemvStages - 1 groups ahead of the MMAs, so every warp keeps
+// several kilobytes in flight without spending registers on them (a thread
+// only reads back what it copied itself: no barrier).  Per group a thread
+// also loads its token's 64 activation bytes (only the lanes whose token
+// exists load) and, every 8 groups, one 16-byte word of 8 scales per row,
+// fetched a batch ahead.  The gate/up projection runs as one matrix of 2I
 // rows with fp32 output (the SwiGLU is applied when the down projection's
 // activations are prepared); the down projection writes bf16 scaled by the
 // row's combine weight.
 constexpr int kGemvWarps = 4;
 constexpr int kGemvRows = 16 * kGemvWarps;  // output rows per block
+constexpr int kGemvStages = 4;
+constexpr size_t kGemvSmem = static_cast<size_t>(kGemvWarps) * kGemvStages * 64 * sizeof(uint4);
 
 template <bool F32OUT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     w4a16_gemv_kernel(const uint4* __restrict__ act16, const int32_t* __restrict__ offsets,
                       const uint8_t* __restrict__ q, const __nv_bfloat16* __restrict__ scales, int N, int K,
                       const float* __restrict__ w_perm, void* __restrict__ out) {
-  constexpr int NM = 1;
+  extern __shared__ uint4 gemv_ring[];
+  constexpr int S = kGemvStages;
   const int e = blockIdx.y;
   const int r_begin = offsets[e], r_end = offsets[e + 1];
   if (r_end <= r_begin) return;
@@ -171,83 +171,79 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
   const int groups = K / 128;
   const size_t rb = static_cast<size_t>(K) / 2;
   const bool batch8 = (groups & 7) == 0;  // scale rows 16-byte aligned every 8 groups
-  const uint8_t* qr[NM][2];
-  const __nv_bfloat16* sr[NM][2];
-#pragma unroll
-  for (int m = 0; m < NM; ++m)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const size_t row = (static_cast<size_t>(e) * NM + m) * N + n0 + 8 * h + g;
-      qr[m][h] = q + row * rb + 16 * t;
-      sr[m][h] = scales + row * groups;
-    }
+  const size_t row0 = static_cast<size_t>(e) * N + n0 + g;
+  const uint8_t* q0 = q + row0 * rb + 16 * t;
+  const uint8_t* q8 = q0 + 8 * rb;
+  const __nv_bfloat16* s0p = scales + row0 * groups;
+  const __nv_bfloat16* s8p = s0p + 8 * groups;
+  uint4* ring = gemv_ring + warp * S * 64 + lane;
+  auto issue = [&](int i) {  // codes of group i (rows g and g+8) into slot i % S
+    uint4* st = ring + (i % S) * 64;
+    cp_async16(st, q0 + static_cast<size_t>(i) * 64);
+    cp_async16(st + 32, q8 + static_cast<size_t>(i) * 64);
+  };
 
   for (int tc = r_begin; tc < r_end; tc += kTok) {
-    __syncwarp();
     const int ntok = min(kTok, r_end - tc);
     const bool has = g < ntok;
     const uint4* ap = act16 + static_cast<size_t>(tc + (has ? g : 0)) * (K / 8) + 4 * t;
-    float acc[NM][4];
 #pragma unroll
-    for (int m = 0; m < NM; ++m)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[m][j] = 0.f;
-    uint4 sv[NM][2], sn[NM][2];
-#pragma unroll
-    for (int m = 0; m < NM; ++m)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        sv[m][h] = sn[m][h] = make_uint4(0, 0, 0, 0);
-        if (batch8) {
-          sv[m][h] = __ldg(reinterpret_cast<const uint4*>(sr[m][h]));
-          if (groups > 8) sn[m][h] = __ldg(reinterpret_cast<const uint4*>(sr[m][h] + 8));
-        }
+    for (int i = 0; i < S - 1; ++i) {
+      if (i < groups) issue(i);
+      cp_async_commit();
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint4 sv0 = make_uint4(0, 0, 0, 0), sv8 = sv0, sn0 = sv0, sn8 = sv0;
+    if (batch8) {
+      sv0 = __ldg(reinterpret_cast<const uint4*>(s0p));
+      sv8 = __ldg(reinterpret_cast<const uint4*>(s8p));
+      if (groups > 8) {
+        sn0 = __ldg(reinterpret_cast<const uint4*>(s0p + 8));
+        sn8 = __ldg(reinterpret_cast<const uint4*>(s8p + 8));
       }
+    }
     for (int g0 = 0; g0 < groups; g0 += 8) {
       if (batch8 && g0 > 0) {
-#pragma unroll
-        for (int m = 0; m < NM; ++m)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            sv[m][h] = sn[m][h];
-            if (g0 + 8 < groups) sn[m][h] = __ldg(reinterpret_cast<const uint4*>(sr[m][h] + g0 + 8));
-          }
+        sv0 = sn0;
+        sv8 = sn8;
+        if (g0 + 8 < groups) {
+          sn0 = __ldg(reinterpret_cast<const uint4*>(s0p + g0 + 8));
+          sn8 = __ldg(reinterpret_cast<const uint4*>(s8p + g0 + 8));
+        }
       }
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const int gq = g0 + jj;
         if (gq < groups) {
-          uint4 cw[NM][2];
-#pragma unroll
-          for (int m = 0; m < NM; ++m)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) cw[m][h] = ld_stream16(qr[m][h] + static_cast<size_t>(gq) * 64);
           uint4 act[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) act[i] = has ? __ldg(ap + gq * 16 + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int m = 0; m < NM; ++m) {
-            float tt[4] = {0.f, 0.f, 0.f, 0.f};
-            tile_group(tt, cw[m][0], cw[m][1], act);
-            float s0, s8;
-            if (batch8) {
-              const uint32_t w0 = (jj >> 1) == 0 ? sv[m][0].x : (jj >> 1) == 1 ? sv[m][0].y : (jj >> 1) == 2 ? sv[m][0].z : sv[m][0].w;
-              const uint32_t w8 = (jj >> 1) == 0 ? sv[m][1].x : (jj >> 1) == 1 ? sv[m][1].y : (jj >> 1) == 2 ? sv[m][1].z : sv[m][1].w;
-              s0 = (jj & 1) ? bf16hi(w0) : bf16lo(w0);
-              s8 = (jj & 1) ? bf16hi(w8) : bf16lo(w8);
-            } else {
-              s0 = bf16_at(sr[m][0] + gq);
-              s8 = bf16_at(sr[m][1] + gq);
-            }
-            acc[m][0] = fmaf(s0, tt[0], acc[m][0]);
-            acc[m][1] = fmaf(s0, tt[1], acc[m][1]);
-            acc[m][2] = fmaf(s8, tt[2], acc[m][2]);
-            acc[m][3] = fmaf(s8, tt[3], acc[m][3]);
+          cp_async_wait<S - 2>();  // group gq has landed
+          if (gq + S - 1 < groups) issue(gq + S - 1);
+          cp_async_commit();
+          const uint4* st = ring + (gq % S) * 64;
+          const uint4 c0 = st[0], c8 = st[32];
+          float tt[4] = {0.f, 0.f, 0.f, 0.f};
+          tile_group(tt, c0, c8, act);
+          float a0, a8;
+          if (batch8) {
+            const uint32_t w0 = (jj >> 1) == 0 ? sv0.x : (jj >> 1) == 1 ? sv0.y : (jj >> 1) == 2 ? sv0.z : sv0.w;
+            const uint32_t w8 = (jj >> 1) == 0 ? sv8.x : (jj >> 1) == 1 ? sv8.y : (jj >> 1) == 2 ? sv8.z : sv8.w;
+            a0 = (jj & 1) ? bf16hi(w0) : bf16lo(w0);
+            a8 = (jj & 1) ? bf16hi(w8) : bf16lo(w8);
+          } else {
+            a0 = bf16_at(s0p + gq);
+            a8 = bf16_at(s8p + gq);
           }
+          acc[0] = fmaf(a0, tt[0], acc[0]);
+          acc[1] = fmaf(a0, tt[1], acc[1]);
+          acc[2] = fmaf(a8, tt[2], acc[2]);
+          acc[3] = fmaf(a8, tt[3], acc[3]);
         }
       }
     }
-    // acc[m][0..1]: row n0 + g, tokens 2t, 2t+1; acc[m][2..3]: row n0 + g + 8
+    cp_async_wait<0>();
+    // acc[0..1]: row n0 + g, tokens 2t, 2t+1; acc[2..3]: row n0 + g + 8
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       const int tok = 2 * t + (cc & 1);
@@ -255,9 +251,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
       if (tok < ntok) {
         const int r = tc + tok;
         if (F32OUT) {
-          static_cast<float*>(out)[static_cast<size_t>(r) * N + col] = acc[0][cc];
+          static_cast<float*>(out)[static_cast<size_t>(r) * N + col] = acc[cc];
         } else {
-          const float v = acc[0][cc] * (w_perm != nullptr ? w_perm[r] : 1.f);
+          const float v = acc[cc] * (w_perm != nullptr ? w_perm[r] : 1.f);
           static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(r) * N + col] = __float2bfloat16_rn(v);
         }
       }
@@ -276,7 +272,7 @@ template <bool F32OUT>
 cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, const void* act16,
                         const int32_t* offsets, const float* w_perm, void* out, cudaStream_t stream) {
   const dim3 grid((N + kGemvRows - 1) / kGemvRows, E);
-  w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, 0, stream>>>(
+  w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, kGemvSmem, stream>>>(
       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
       static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out);
   return cudaGetLastError();
