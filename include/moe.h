@@ -236,6 +236,19 @@ MOE_API moe_status moe_permute_no_alloc(const moe_config* cfg, const int32_t* to
  * debugging. */
 MOE_API moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t* code);
 
+/* Test hook for the device-timeout path; the pages have no counterpart (it
+ * checks this library's own failure handling).  Zeroes `scratch` (device,
+ * 256-byte aligned, at least MOE_SELFTEST_SCRATCH_BYTES) and launches the
+ * split-K tensor-core GEMM on one 128 x 16 x 64 tile of zero operands held
+ * in it, with the signal that the tile's MMAs finished withheld and every
+ * wait limited to 20 ms.  The epilogue's wait runs out, the kernel records
+ * MOE_ERR_DEVICE_TIMEOUT in scratch's error word, drains its own copy and
+ * MMAs, frees its tensor memory and exits; the context stays usable.  Read
+ * the result with moe_read_device_error(scratch, ...).  Returns MOE_OK once
+ * the launch is enqueued. */
+#define MOE_SELFTEST_SCRATCH_BYTES 65536
+MOE_API moe_status moe_selftest_device_timeout(void* scratch, size_t scratch_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

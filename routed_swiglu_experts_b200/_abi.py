@@ -31,9 +31,10 @@ MOE_MAX_EXPERTS = 1024
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",
     "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward",
-    "moe_read_device_error", "moe_permute_no_alloc",
+    "moe_read_device_error", "moe_permute_no_alloc", "moe_selftest_device_timeout",
 )
 MOE_NO_ALLOC_MAX_ROWS = 131072
+MOE_SELFTEST_SCRATCH_BYTES = 65536
 
 
 class MoEError(RuntimeError):
@@ -95,6 +96,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_combine": (ctypes.c_int, [CFG, P, P, P, P, I32, P, P]),
         "moe_forward": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, SZ, P]),
         "moe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
+        "moe_selftest_device_timeout": (ctypes.c_int, [P, SZ, P]),
         "moe_permute_no_alloc": (ctypes.c_int, [CFG, P, P, P, I32, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -209,6 +211,14 @@ def moe_read_device_error(ws, stream=None) -> int:
     _check(load_library().moe_read_device_error(_ptr(ws), _stream(stream), ctypes.byref(code)),
            "moe_read_device_error")
     return code.value
+
+
+def moe_selftest_device_timeout(scratch, stream=None):
+    """Test hook: force the tensor-core kernel's timeout path on a tiny tile
+    (the error lands in scratch's error word; read it with
+    moe_read_device_error(scratch))."""
+    _check(load_library().moe_selftest_device_timeout(_ptr(scratch), scratch.numel() * scratch.element_size(),
+                                                      _stream(stream)), "moe_selftest_device_timeout")
 
 
 def status_strings():

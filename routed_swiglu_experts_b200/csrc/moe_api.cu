@@ -335,6 +335,13 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out, stream));
 }
 
+moe_status moe_selftest_device_timeout(void* scratch, size_t scratch_bytes, moe_stream_t stream) {
+  if (scratch == nullptr || scratch_bytes < MOE_SELFTEST_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(cudaMemsetAsync(scratch, 0, MOE_SELFTEST_SCRATCH_BYTES, stream));
+  return from_cuda(launch_splitk_timeout_selftest(scratch, err_word(scratch), stream));
+}
+
 moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t* code) {
   if (ws == nullptr || code == nullptr) return MOE_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;

@@ -39,6 +39,7 @@ size_t router_topk_smem(int E);
 cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, int parts, int N, int n_mma,
                                int k_splits, float* part, int32_t* err, int num_sms, cudaStream_t stream);
 int splitk_actual_splits(int K, int parts, int k_splits);
+cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStream_t stream);
 int router_actual_splits(int H, int k_splits);
 cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
                                int32_t* err, int num_sms, cudaStream_t stream);

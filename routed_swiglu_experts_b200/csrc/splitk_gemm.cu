@@ -53,6 +53,8 @@ struct alignas(64) SplitKParams {
   int32_t n_tiles;            // output-column tiles x k_splits
   uint32_t idesc;             // MMA instruction descriptor
   int32_t* err;
+  uint64_t timeout_ns;        // limit of every wait on another role's progress
+  int32_t test_withhold;      // test hook: never signal the first tile's accumulator
 };
 
 struct SmemCtl {
@@ -151,7 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         tile_k_range(P, ti, kb0, kb1);
         const uint32_t stage_tx = static_cast<uint32_t>(A_BYTES + P.n_mma * BK * 2);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.timeout_ns)) {
             fail(1);
             ok = false;
             break;
@@ -191,14 +193,14 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         const uint32_t idesc = P.idesc;
         int kb0, kb1;
         tile_k_range(P, ti, kb0, kb1);
-        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, P.timeout_ns)) {
           fail(2);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, P.timeout_ns)) {
             fail(3);
             ok = false;
             break;
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
           }
         }
         if (!ok) break;
-        umma_commit(&c.tmem_full[acc]);
+        if (!(P.test_withhold && t == static_cast<int>(blockIdx.x))) umma_commit(&c.tmem_full[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
       const int ncol0 = ti.nidx * P.n_mma;
       // every lane waits; the outcome is made warp-uniform before the
       // warp-collective TMEM loads
-      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
+      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, P.timeout_ns);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) fail(4);
         break;
@@ -334,10 +336,44 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   P.n_tiles = ((N + n_mma - 1) / n_mma) * P.k_splits;
   P.idesc = umma_idesc_bf16(BM, n_mma);
   P.err = err;
+  P.timeout_ns = kTimeoutNs;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   const int tiles = ((rows + BM - 1) / BM) * P.n_tiles;
   splitk_gemm_kernel<<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
+  return cudaGetLastError();
+}
+
+// Test hook: one 128 x 16 x 64 tile over zero operands in `scratch` whose
+// MMA completion is never signalled to the epilogue, with a 20 ms wait limit.
+// The epilogue's wait runs out, records MOE_ERR_DEVICE_TIMEOUT (detail 4) in
+// *err, and every role leaves through the normal drain: the producer waits
+// for its copy, the MMA issuer for its MMAs, TMEM is freed.
+cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStream_t stream) {
+  unsigned char* base = static_cast<unsigned char*>(scratch);
+  void* a = base + 1024;                   // bf16 [128, 64]
+  void* b = base + 1024 + 128 * 64 * 2;    // bf16 [16, 64]
+  float* part = reinterpret_cast<float*>(base + 1024 + 128 * 64 * 2 + 16 * 64 * 2);  // fp32 [128, 16]
+  SplitKParams P;
+  memset(&P, 0, sizeof(P));
+  if (!encode_a(&P.tma_a, a, 128, 64)) return cudaErrorInvalidValue;
+  if (!encode_b(&P.tma_b, b, 1, 16, 64, 16)) return cudaErrorInvalidValue;
+  P.out_f32 = part;
+  P.rows = 128;
+  P.n_out = 16;
+  P.n_mma = 16;
+  P.k_blocks = 1;
+  P.parts = 1;
+  P.kb_per_split = 1;
+  P.k_splits = 1;
+  P.n_tiles = 1;
+  P.idesc = umma_idesc_bf16(BM, 16);
+  P.err = err;
+  P.timeout_ns = 20000000ull;
+  P.test_withhold = 1;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  splitk_gemm_kernel<<<1, THREADS, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 

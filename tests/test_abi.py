@@ -173,3 +173,11 @@ def _load_fresh(path):
         return _abi.load_library(path)
     finally:
         _abi._lib = saved
+
+
+def test_selftest_timeout_argument_checks(lib):
+    """The timeout test hook validates its scratch before touching the GPU."""
+    n = _abi.MOE_SELFTEST_SCRATCH_BYTES
+    assert lib.moe_selftest_device_timeout(None, n, None) == _abi.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_device_timeout(FAKE, n - 1, None) == _abi.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_device_timeout(FAKE + 16, n, None) == _abi.MOE_ERR_INVALID_ARG
