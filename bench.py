@@ -347,9 +347,10 @@ def bench_ours(args, rank, world, local_rank):
     if c.w4a16:
         touched, nbytes = w4a16_bytes(c, ids.cpu())
         achieved = nbytes / ffn_s / 1e9
-        roof = {"kernel": "W4A16 expert FFN (register-dequant gate/up+SwiGLU and down launches) + bf16 "
-                          "shared expert", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+        roof = {"kernel": "W4A16 expert FFN (register-dequant gate/up and down GEMV launches with their "
+                          "activation preps) + bf16 shared expert", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": traffic_from_profile(f"grouped_ffn_{c.name}"),
                 "peak_source": f"{peaks['source']} HBM copy", "bytes_per_call": nbytes,
                 "touched_experts": touched}
     else:

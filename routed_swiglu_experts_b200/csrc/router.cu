@@ -130,8 +130,19 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     const int w = idx / E, e = idx - w * E;
     const int tt = t0 + w;
     if (tt < T) {
+      // slices are added in ascending order, loaded 8 at a time
       float l = 0.f;
-      for (int ks = 0; ks < KS; ++ks) l += part[(static_cast<size_t>(ks) * T + tt) * E + e];
+      const float* pp = part + static_cast<size_t>(tt) * E + e;
+      const size_t slice = static_cast<size_t>(T) * E;
+      int ks = 0;
+      for (; ks + 8 <= KS; ks += 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __ldg(pp + (ks + j) * slice);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) l += v[j];
+      }
+      for (; ks < KS; ++ks) l += __ldg(pp + ks * slice);
       const float sv = 1.f / (1.f + expf(-l));
       float* sw = reinterpret_cast<float*>(smem_raw + pw * w + static_cast<size_t>(E) * 8);
       sw[e] = sv;
