@@ -160,28 +160,34 @@ def gemm_flops(cfg):
     return routed, shared
 
 
-def run_cpu_baseline(inp, passes=3):
+def run_cpu_baseline(inp, min_seconds=10.0, max_passes=20):
+    """The oracle as it stands, on the host cores: whole-layer passes until
+    about `min_seconds` of CPU work (at least one, at most `max_passes`)."""
     import torch
     import oracle
     cores = torch.get_num_threads()
     t0 = time.perf_counter()
-    for _ in range(passes):
+    passes = 0
+    while passes < max_passes:
         oracle.moe_forward(inp)
+        passes += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
     dt = time.perf_counter() - t0
     return {"value": passes * inp.cfg.T / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{passes} passes of the full mid layer ({inp.cfg.T} tokens each), fp64 torch CPU, "
+            "sample": f"{passes} passes of the full {inp.cfg.name} layer ({inp.cfg.T} tokens each), fp64 torch CPU, "
                       f"{dt:.1f} s"}
 
 
 def w4a16_bytes(cfg, ids):
-    """HBM bytes one W4A16 decode call must move: codes + scales of every
-    touched expert, the bf16 shared expert, router weight, activations."""
+    """HBM bytes the W4A16 expert FFN call must move: codes + scales of every
+    touched expert, the bf16 shared expert, and its activations (x_perm and
+    x read, y_perm and the shared output written)."""
     touched = int(len(set(ids.reshape(-1).tolist())))
     per_expert = (2 * cfg.I * cfg.H // 2 + cfg.H * cfg.I // 2) + 2 * (2 * cfg.I * cfg.H // 128 + cfg.H * cfg.I // 128)
     shared = 2 * (2 * cfg.I_s * cfg.H + cfg.H * cfg.I_s)
-    router = 4 * cfg.E * cfg.H
     acts = 2 * cfg.T * cfg.H * (2 + 2 * cfg.k)
-    return touched, touched * per_expert + shared + router + acts
+    return touched, touched * per_expert + shared + acts
 
 
 def launches_per_step(cfg):
@@ -189,7 +195,7 @@ def launches_per_step(cfg):
     logits, top-k), permute 3 (count/rank, scan, scatter), combine 1, plus the
     expert FFN path."""
     n = 7
-    small_shared = cfg.I_s > 0 and cfg.T <= 32 and cfg.H % 32 == 0 and cfg.I_s % 32 == 0
+    small_shared = cfg.I_s > 0 and cfg.T <= 32  # split-K GEMMs + slice sums for the shared expert
     shared = (4 if small_shared else 2) if cfg.I_s > 0 else 0
     if cfg.w4a16:
         n += 4 + shared          # routed: (prep + gemv) x 2
