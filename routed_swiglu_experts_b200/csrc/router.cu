@@ -80,6 +80,7 @@ __device__ __forceinline__ void exact_biased_pair(const __nv_bfloat16* __restric
   const float* w0r = wr + static_cast<size_t>(e0) * H;
   const float* w1r = wr + static_cast<size_t>(e1) * H;
   double a0 = 0.0, a1 = 0.0;
+#pragma unroll 4
   for (int h = lane * 8; h < H; h += 256) {
     const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + h));
     const float4 p0 = __ldg(reinterpret_cast<const float4*>(w0r + h));
@@ -105,7 +106,30 @@ __device__ __forceinline__ void exact_biased_pair(const __nv_bfloat16* __restric
   b1 = 1.0 / (1.0 + exp(-a1)) + (bias != nullptr ? static_cast<double>(bias[e1]) : 0.0);
 }
 
-// One warp per token.
+// Single-expert form of exact_biased_pair (same per-lane summation order).
+__device__ __forceinline__ double exact_biased_one(const __nv_bfloat16* __restrict__ xr,
+                                                   const float* __restrict__ wr, const float* __restrict__ bias,
+                                                   int H, int lane, int e0) {
+  const float* w0r = wr + static_cast<size_t>(e0) * H;
+  double a0 = 0.0;
+#pragma unroll 4
+  for (int h = lane * 8; h < H; h += 256) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + h));
+    const float4 p0 = __ldg(reinterpret_cast<const float4*>(w0r + h));
+    const float4 p1 = __ldg(reinterpret_cast<const float4*>(w0r + h + 4));
+    const double xv8[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
+                           bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+    const float pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a0 = fma(xv8[j], static_cast<double>(pw[j]), a0);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+  return 1.0 / (1.0 + exp(-a0)) + (bias != nullptr ? static_cast<double>(bias[e0]) : 0.0);
+}
+
+// One warp per token (with one token per block, every warp of the block
+// shares that token's fp64 scores).
 //  1. s = sigmoid(sum of the partial logits), b = s + bias (fp32).
 //  2. Extract experts in (b desc, id asc) order: the top k+1, and, while the
 //     k-th/(k+1)-th boundary is a near-tie, every further expert that
@@ -150,10 +174,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     }
   }
   __syncthreads();
-  const int t = t0 + warp;
-  if (warp >= tpb || t >= T) return;
+  const bool coop = tpb == 1;  // block-uniform
+  const int t = t0 + (coop ? 0 : warp);
+  if (coop ? t >= T : (warp >= tpb || t >= T)) return;
+  const bool owner = !coop || warp == 0;
 
-  unsigned char* base = smem_raw + pw * warp;
+  unsigned char* base = smem_raw + pw * (coop ? 0 : warp);
   double* v64 = reinterpret_cast<double*>(base);
   float* s_sm = reinterpret_cast<float*>(base + static_cast<size_t>(E) * 8);
   float* b_sm = s_sm + E;
@@ -162,9 +188,11 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   int* res = lst + E;
   const int nm = (E + 31) / 32;  // entries per lane: e = lane + 32 m
 
-  // 2. ordered extraction
-  uint32_t taken = 0;
+  // 2. ordered extraction (the owner warp)
+  __shared__ int s_n;
   int n = 0;
+  if (owner) {
+  uint32_t taken = 0;
   const int k1 = min(k + 1, E);
   while (n < E) {
     float v = -INFINITY;
@@ -193,22 +221,49 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     ++n;
   }
   if (lane < k) res[lane] = lst[lane];
+  if (coop && lane == 0) s_n = n;
   __syncwarp();
+  }
 
-  // 3. fp64 re-order of the near-tie clusters that reach into the top k
+  // 3. fp64 re-order of the near-tie clusters that reach into the top k.
+  //    Cluster [a, b]: a maximal run of adjacent gaps below tau starting at
+  //    a < k.  With one token per block all warps first compute the fp64
+  //    scores of every clustered entry, then the owner orders them.
   const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+  if (coop) {
+    __syncthreads();
+    n = s_n;
+    for (int i = warp; i < n; i += kTopkWarps) {
+      // entry i needs an fp64 score if its cluster has two entries or more
+      int a = 0, b = 0;
+      while (true) {
+        b = a;
+        while (b + 1 < n && lv[b] - lv[b + 1] < tau) ++b;
+        if (i <= b || b + 1 >= k) break;
+        a = b + 1;
+      }
+      if (a < k && i >= a && i <= b && b > a) {
+        const double d = exact_biased_one(xr, wr, bias, H, lane, lst[i]);
+        if (lane == 0) v64[i] = d;
+      }
+    }
+    __syncthreads();
+    if (!owner) return;
+  }
   int a = 0;
   while (a < k) {
     int b = a;
     while (b + 1 < n && lv[b] - lv[b + 1] < tau) ++b;
     if (b > a) {
-      for (int i = a; i <= b; i += 2) {
-        const int j = min(i + 1, b);
-        double d0, d1;
-        exact_biased_pair(xr, wr, bias, H, lane, lst[i], lst[j], d0, d1);
-        if (lane == 0) {
-          v64[i] = d0;
-          v64[j] = d1;
+      if (!coop) {
+        for (int i = a; i <= b; i += 2) {
+          const int j = min(i + 1, b);
+          double d0, d1;
+          exact_biased_pair(xr, wr, bias, H, lane, lst[i], lst[j], d0, d1);
+          if (lane == 0) {
+            v64[i] = d0;
+            v64[j] = d1;
+          }
         }
       }
       __syncwarp();
@@ -258,6 +313,7 @@ RouterPlan router_plan(int T, int E, int H) {
   int ks = (148 + tiles0 - 1) / tiles0;          // about one wave of CTAs
   ks = std::min(ks, std::max(1, total_kb / 4));  // at least 4 k-blocks per split
   ks = std::min(ks, std::max(1, kRouterPartialRows / std::max(T, 1)));
+  ks = std::min(ks, 32);  // the top-k kernel adds every slice: keep its reads short
   p.ks = router_actual_splits(H, std::max(ks, 1));
   return p;
 }

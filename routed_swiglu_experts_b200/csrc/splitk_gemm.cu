@@ -53,6 +53,7 @@ struct alignas(64) SplitKParams {
   int32_t n_tiles;            // output-column tiles x k_splits
   uint32_t idesc;             // MMA instruction descriptor
   int32_t* err;
+  int32_t a_box_rows;         // rows per A copy: 128, or fewer when A has fewer rows
   uint64_t timeout_ns;        // limit of every wait on another role's progress
   int32_t test_withhold;      // test hook: never signal the first tile's accumulator
 };
@@ -151,7 +152,9 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         const int ncol0 = ti.nidx * P.n_mma;
         int kb0, kb1;
         tile_k_range(P, ti, kb0, kb1);
-        const uint32_t stage_tx = static_cast<uint32_t>(A_BYTES + P.n_mma * BK * 2);
+        // A rows past a_box_rows stay stale in shared memory: they only feed
+        // accumulator rows that are never stored
+        const uint32_t stage_tx = static_cast<uint32_t>((P.a_box_rows + P.n_mma) * BK * 2);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.timeout_ns)) {
             fail(1);
@@ -298,10 +301,10 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
 // ------------------------------------------------------------------ host --
 
 // 2-D bf16 map over [rows, K] (K innermost), box 64 x 128, 128-byte swizzle.
-bool encode_a(CUtensorMap* m, const void* base, int rows, int K) {
+bool encode_a(CUtensorMap* m, const void* base, int rows, int K, int box_rows = BM) {
   const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {BK, BM};
+  const uint32_t box[2] = {BK, static_cast<uint32_t>(box_rows)};
   return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -321,7 +324,10 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   if (n_mma < 16 || n_mma > 256 || n_mma % 16 != 0 || parts < 1) return cudaErrorInvalidValue;
   SplitKParams P;
   memset(&P, 0, sizeof(P));
-  if (!encode_a(&P.tma_a, a, rows, K)) return cudaErrorInvalidValue;
+  // a single row tile with few rows copies only a multiple of 8 rows of it
+  const int a_box = rows < BM ? std::max(8, (rows + 7) / 8 * 8) : BM;
+  if (!encode_a(&P.tma_a, a, rows, K, a_box)) return cudaErrorInvalidValue;
+  P.a_box_rows = a_box;
   if (!encode_b(&P.tma_b, b, parts, N, K, n_mma)) return cudaErrorInvalidValue;
   P.out_f32 = part;
   P.rows = rows;
@@ -357,6 +363,7 @@ cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStre
   SplitKParams P;
   memset(&P, 0, sizeof(P));
   if (!encode_a(&P.tma_a, a, 128, 64)) return cudaErrorInvalidValue;
+  P.a_box_rows = BM;
   if (!encode_b(&P.tma_b, b, 1, 16, 64, 16)) return cudaErrorInvalidValue;
   P.out_f32 = part;
   P.rows = 128;
