@@ -197,7 +197,9 @@ def launches_per_step(cfg):
     n = 7
     small_shared = cfg.I_s > 0 and cfg.T <= 32  # split-K GEMMs + slice sums for the shared expert
     shared = (4 if small_shared else 2) if cfg.I_s > 0 else 0
-    if cfg.w4a16:
+    if cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E:
+        n += 3 + shared          # routed: token prep + dequantising gate/up and down GEMMs
+    elif cfg.w4a16:
         n += 4 + shared          # routed: (prep + gemv) x 2
     else:
         n += 2 + (4 if small_shared else 0)  # routed + large shared share two launches
@@ -350,7 +352,7 @@ def bench_ours(args, rank, world, local_rank):
     peaks = measured_peaks()
     routed_f, shared_f = gemm_flops(c)
     ffn_s = stage_ms["grouped_ffn"] / 1e3
-    if c.w4a16:
+    if c.w4a16 and c.T * c.k < 32 * c.E:  # the GEMV path: HBM-bound
         touched, nbytes = w4a16_bytes(c, ids.cpu())
         achieved = nbytes / ffn_s / 1e9
         roof = {"kernel": "W4A16 expert FFN (register-dequant gate/up and down GEMV launches with their "
@@ -361,7 +363,9 @@ def bench_ours(args, rank, world, local_rank):
                 "touched_experts": touched}
     else:
         achieved = (routed_f + shared_f) / ffn_s / 1e12
-        roof = {"kernel": "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
+        roof = {"kernel": ("grouped W4A16 FFN (int4 dequantised to fp16 in shared memory, tcgen05 gate/up+SwiGLU "
+                           "and down+weight launches) + bf16 shared expert") if c.w4a16 else
+                          "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
                           "routed + shared expert)",
                 "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],

@@ -57,4 +57,10 @@ DECODE_W4A16 = LayerConfig("decode_w4a16", T=32, H=6144, E=256, k=8, I=2048,
                            I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
                            w4a16=True)
 
-CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16)}
+# Not one of the five benchmark layers: the large prefill shape with the
+# decode layer's int4 group-128 expert weights, for the grouped W4A16 GEMM.
+PREFILL_W4A16 = LayerConfig("prefill_w4a16", T=16384, H=6144, E=256, k=8, I=2048,
+                            I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
+                            w4a16=True)
+
+CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16, PREFILL_W4A16)}

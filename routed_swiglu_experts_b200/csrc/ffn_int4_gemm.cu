@@ -1,0 +1,667 @@
+// Grouped W4A16 expert FFN GEMMs for many tokens per expert, on CTA pairs
+// (tcgen05.mma.cta_group::2, fp16 operands, fp32 accumulate).
+//
+// "Module glm5next_mlp", W4A16 grouped prefill GEMM (MOE_GROUPED_MODULE with
+// int4 group-128 weights, w = (q - 8) * scale): one launch per projection
+// for all experts, driven by the expert row offsets.
+//   gate/up:  h[t, f] = silu(min(G, L)) * clamp(U, -L, L), rounded to bf16
+//             (§Numerics: asymmetric clamp), stored as fp16 for the down MMA
+//   down:     y[t, n] = bf16( row_scale[t] * sum_i W_d[n, i] h[t, i] )
+//
+// Same tile and roles as the bf16 CTA-pair kernel (weights = M, 256 rows per
+// pair; tokens = N rounded to 16; two 256-column TMEM accumulators), plus
+// four dequantisation warps per CTA: TMA copies the int4 codes of the CTA's
+// 128 weight rows (32 bytes per row per 64-deep K step) into a staging ring;
+// each dequantisation thread turns one row's 64 codes into fp16 weights
+//   (q - 8) * scale   -- exact in fp16: a 4-bit integer times a bf16 scale
+// and writes them, 128-byte swizzled, into the MMA's A stage, then the warp
+// arrives on the pair's full barrier.  Within every aligned 8 of K the
+// weights sit in the order {0, 4, 1, 5, 2, 6, 3, 7} (how four LOP3s split a
+// 32-bit code word); the tokens are prepared in the same order, and the
+// gate/up epilogue writes h in it, so the K sum is unchanged.
+// Every mbarrier wait is bounded (MOE_ERR_DEVICE_TIMEOUT on expiry).
+#include <cstring>
+
+#include <cuda_fp16.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BK = 64;
+constexpr int ROWS = 128;                    // weight rows per CTA
+constexpr int TOK = 256;                     // tokens per pair tile
+constexpr int STAGES = 5;                    // A (dequantised) and B (token) stages
+constexpr int CKB = 4;                       // 64-deep K steps per code copy (128-byte code rows)
+constexpr int CSTAGES = 2;                   // code stages
+constexpr int A_BYTES = ROWS * BK * 2;       // 16 KB fp16 weights (dequantised)
+constexpr int B_BYTES = (TOK / 2) * BK * 2;  // 16 KB fp16 tokens (this CTA's half)
+constexpr int C_BYTES = ROWS * CKB * BK / 2; // 16 KB int4 codes, 128-byte swizzled rows
+constexpr int DQ_WARPS = 8;                  // dequantisation warps: two threads per weight row
+constexpr int DQ_WARP0 = 7;                  // first dequantisation warp
+constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;  // 0-3 epilogue, 4 token TMA, 5 MMA, 6 code TMA, 7.. dequant
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr int HPITCH = 144;                  // bytes per token row of the staged gate/up output
+
+enum class Kind { GateUp, Down };
+
+struct alignas(64) Int4Params {
+  CUtensorMap tma_q;          // codes: gate/up {K/2, 8, 2, N/8, G} box {128, 8, 2, 8, 1}; down {K/2, N, G} box {128, 128, 1}
+  CUtensorMap tma_x;          // fp16 tokens {K, rows} box {64, 128}, 128-byte swizzle
+  const int32_t* offsets;     // [groups + 1]
+  const __nv_bfloat16* scales;  // gate/up [G, 2N, K/128]; down [G, N, K/128]
+  void* out;                  // gate/up: fp16 h [rows, N]; down: bf16 y [rows, N]
+  const float* row_scale;     // down: per token row (or nullptr)
+  int32_t groups;
+  int32_t rows;
+  int32_t n_out;              // N: I (gate/up) or H (down)
+  int32_t K;
+  int32_t k_blocks;
+  int32_t f_tiles;
+  float limit;
+  int32_t* err;
+};
+
+struct Ctl {
+  uint64_t full[STAGES];      // pair's first CTA: the dequantisation warps of both CTAs
+  uint64_t tok_full[STAGES];  // pair's first CTA: token bytes of both CTAs
+  uint64_t empty[STAGES];
+  uint64_t code_full[CSTAGES];   // this CTA's codes landed
+  uint64_t code_empty[CSTAGES];  // this CTA's dequantisation warps read them
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+  int32_t tiles;
+  int32_t off[MOE_MAX_EXPERTS + 1];
+  int32_t tp[MOE_MAX_EXPERTS + 1];
+  uint4 obuf[512];
+};
+
+constexpr size_t kSmem = 1024 + STAGES * (A_BYTES + B_BYTES) + CSTAGES * C_BYTES + sizeof(Ctl);
+static_assert(kSmem <= 232448, "fits the 227 KB opt-in shared memory");
+
+struct Tile {
+  int g, fidx, row0, ntok, nmma;
+};
+
+__device__ __forceinline__ Tile decode(const Int4Params& P, const Ctl& c, int t) {
+  Tile ti;
+  const int nf = P.f_tiles;
+  const int u = t / nf;
+  int lo = 0, hi = P.groups;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (c.tp[mid] <= u) lo = mid; else hi = mid;
+  }
+  ti.g = lo;
+  const int tm = c.tp[lo + 1] - c.tp[lo];
+  const int local = t - c.tp[lo] * nf;
+  ti.fidx = local / tm;
+  const int tmi = local - ti.fidx * tm;
+  ti.row0 = c.off[lo] + tmi * TOK;
+  ti.ntok = min(TOK, c.off[lo + 1] - ti.row0);
+  ti.nmma = (ti.ntok + 15) / 16 * 16;
+  return ti;
+}
+
+__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// One code word (8 codes, k = 0..7 of an aligned 8) -> four fp16x2 weights in
+// the order {k0, k4}, {k1, k5}, {k2, k6}, {k3, k7}.  The fp16 exponent OR
+// gives 1024 + q (low nibble of each half) or 1024 + 16 q (high nibble);
+// subtracting 1032 or 1152 leaves q - 8 or 16 (q - 8) exactly, and the scale
+// (s, or s / 16 for the 16-times values) makes the weight; every step is
+// exact in fp16.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t s2_16) {
+  const uint32_t w8 = w >> 8;
+  uint4 r;
+  r.x = hmul2_u(hsub2_u((w & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
+  r.y = hmul2_u(hsub2_u((w & 0x00F000F0u) | 0x64006400u, 0x64806480u), s2_16);
+  r.z = hmul2_u(hsub2_u((w8 & 0x000F000Fu) | 0x64006400u, 0x64086408u), s2);
+  r.w = hmul2_u(hsub2_u((w8 & 0x00F000F0u) | 0x64006400u, 0x64806480u), s2_16);
+  return r;
+}
+
+// Position of feature f inside its aligned 8 after the {0,4,1,5,2,6,3,7} order.
+__device__ __forceinline__ int slot_of(int f) {
+  const int j = f & 7;
+  return (f & ~7) | ((j & 3) * 2 + (j >> 2));
+}
+
+template <Kind KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    ffn_int4_pair_kernel(const __grid_constant__ Int4Params P) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  unsigned char* smem_a = smem;
+  unsigned char* smem_b = smem + STAGES * A_BYTES;
+  unsigned char* smem_c = smem_b + STAGES * B_BYTES;
+  Ctl& c = *reinterpret_cast<Ctl*>(smem_c + CSTAGES * C_BYTES);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&c.full[s], 2 * DQ_WARPS);
+      mbar_init(&c.tok_full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int s = 0; s < CSTAGES; ++s) {
+      mbar_init(&c.code_full[s], 1);
+      mbar_init(&c.code_empty[s], DQ_WARPS);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&c.tmem_full[a], 1);
+      mbar_init(&c.tmem_empty[a], 2 * 4);
+    }
+    mbar_init(&c.mma_done, 1);
+    c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&P.tma_q);
+    tma_prefetch_desc(&P.tma_x);
+  }
+  if (warp == 0) {  // offsets + token-tile prefix per expert
+    const int G = P.groups;
+    const int per = (G + 31) / 32;
+    int local = 0;
+    for (int j = 0; j < per; ++j) {
+      const int g = lane * per + j;
+      if (g < G) {
+        const int o0 = P.offsets[g], o1 = P.offsets[g + 1];
+        c.off[g] = o0;
+        local += (o1 - o0 + TOK - 1) / TOK;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int j = 0; j < per; ++j) {
+      const int g = lane * per + j;
+      if (g < G) {
+        c.tp[g] = run;
+        run += (P.offsets[g + 1] - P.offsets[g] + TOK - 1) / TOK;
+      }
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) {
+      c.off[G] = P.offsets[G];
+      c.tp[G] = total;
+      c.tiles = total * P.f_tiles;
+    }
+  }
+  if (warp == 5) tmem_alloc_pair(&c.tmem_base, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+
+  const uint32_t tmem_base = c.tmem_base;
+  const int total_tiles = c.tiles;
+  volatile int32_t* abort_flag = &c.abort_flag;
+  auto fail = [&](int detail) {
+    *abort_flag = 1;
+    report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, detail);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        const Tile ti = decode(P, c, t);
+        const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
+        for (int kb = 0; kb < P.k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+            fail(41);
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&c.tok_full[stage], 2 * B_BYTES);
+          tma_load_2d_pair(smem_b + stage * B_BYTES, &P.tma_x, kb * BK, xrow, leader_bar(&c.tok_full[stage]));
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // drain (first CTA): the last token copies of both CTAs complete on
+      // its tok_full barriers
+      const int nst = issued < STAGES ? issued : STAGES;
+      for (int j = 0; j < nst; ++j) {
+        const int i = issued - 1 - j;
+        volatile int32_t never = 0;
+        if (leader && !mbar_wait_bounded(&c.tok_full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1), &never,
+                                         kTimeoutNs))
+          report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, 48);
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------- MMA issuer (first CTA) --
+    if (leader && lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        const Tile ti = decode(P, c, t);
+        const uint32_t idesc = umma_idesc_f16(2 * ROWS, ti.nmma);
+        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          fail(42);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < P.k_blocks; ++kb) {
+          if (!mbar_wait_bounded(&c.tok_full[stage], phase, abort_flag, kTimeoutNs) ||
+              !mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
+            fail(43);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem_a + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(smem_b + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&c.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&c.tmem_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      umma_commit_pair_leader(&c.mma_done);
+      volatile int32_t never = 0;
+      if (!mbar_wait_bounded(&c.mma_done, 0, &never, kTimeoutNs)) report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, 47);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------- code TMA producer --
+    if (lane == 0) {
+      int cs = 0, issued = 0;
+      uint32_t cphase = 0;
+      bool ok = true;
+      const int ncb = (P.k_blocks + CKB - 1) / CKB;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        const Tile ti = decode(P, c, t);
+        for (int cb = 0; cb < ncb; ++cb) {
+          if (!mbar_wait_bounded(&c.code_empty[cs], cphase ^ 1u, abort_flag, kTimeoutNs)) {
+            fail(46);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&c.code_full[cs], C_BYTES);
+          unsigned char* sc = smem_c + cs * C_BYTES;
+          if (KIND == Kind::GateUp) {
+            const int fb = ti.fidx * 16 + static_cast<int>(rank) * 8;  // first 8-feature block
+            tma_load_5d(sc, &P.tma_q, cb * (CKB * BK / 2), 0, 0, fb, ti.g, &c.code_full[cs]);
+          } else {
+            const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
+            tma_load_3d(sc, &P.tma_q, cb * (CKB * BK / 2), n, ti.g, &c.code_full[cs]);
+          }
+          ++issued;
+          if (++cs == CSTAGES) {
+            cs = 0;
+            cphase ^= 1u;
+          }
+        }
+      }
+      // drain: the last code copy of each stage
+      const int nst = issued < CSTAGES ? issued : CSTAGES;
+      for (int j = 0; j < nst; ++j) {
+        const int i = issued - 1 - j;
+        volatile int32_t never = 0;
+        if (!mbar_wait_bounded(&c.code_full[i % CSTAGES], static_cast<uint32_t>((i / CSTAGES) & 1), &never,
+                               kTimeoutNs))
+          report_error(P.err, MOE_ERR_DEVICE_TIMEOUT, 49);
+      }
+    }
+  } else if (warp >= DQ_WARP0) {
+    // ------------------------------------- dequantisation (warps 7 .. 14) --
+    // thread -> (weight row i of this CTA's 128, half of the row's 64 codes)
+    const int dq = threadIdx.x - DQ_WARP0 * 32;
+    const int i = dq & (ROWS - 1), half = dq / ROWS;
+    const int groups = P.K / 128;
+    const bool batch8 = (groups & 7) == 0;  // the row's scales come 8 groups per 16-byte load
+    const uint32_t full_leader = leader_bar(&c.full[0]);
+    int stage = 0, cs = 0;
+    uint32_t phase = 0, cphase = 0;
+    for (int t = pair; t < total_tiles; t += npairs) {
+      const Tile ti = decode(P, c, t);
+      // this row's scales (nullptr: past the end of the matrix, codes are zero-filled)
+      const __nv_bfloat16* sp = nullptr;
+      if (KIND == Kind::GateUp) {
+        const int f = ti.fidx * 128 + static_cast<int>(rank) * 64 + (i >> 4) * 8 + (i & 7);
+        const int u = (i >> 3) & 1;
+        if (f < P.n_out)
+          sp = P.scales + (static_cast<size_t>(ti.g) * 2 * P.n_out + static_cast<size_t>(u) * P.n_out + f) * groups;
+      } else {
+        const int n = ti.fidx * 256 + static_cast<int>(rank) * 128 + i;
+        if (n < P.n_out) sp = P.scales + (static_cast<size_t>(ti.g) * P.n_out + n) * groups;
+      }
+      uint4 sv = make_uint4(0, 0, 0, 0), sn = sv;
+      if (batch8 && sp != nullptr) {
+        sv = __ldg(reinterpret_cast<const uint4*>(sp));
+        if (groups > 8) sn = __ldg(reinterpret_cast<const uint4*>(sp + 8));
+      }
+      bool ok = true;
+      for (int kb = 0; kb < P.k_blocks; ++kb) {
+        const int gq = kb >> 1;
+        if (batch8 && (kb & 15) == 0 && kb > 0) {  // next batch of 8 groups
+          sv = sn;
+          if (sp != nullptr && gq + 8 < groups) sn = __ldg(reinterpret_cast<const uint4*>(sp + gq + 8));
+        }
+        float sf = 0.f;
+        if (sp != nullptr) {
+          if (batch8) {
+            const int j = gq & 7;
+            const uint32_t wv = (j >> 1) == 0 ? sv.x : (j >> 1) == 1 ? sv.y : (j >> 1) == 2 ? sv.z : sv.w;
+            sf = (j & 1) ? bf16hi(wv) : bf16lo(wv);
+          } else {
+            sf = __bfloat162float(sp[gq]);
+          }
+        }
+        const __half2 s2h = __floats2half2_rn(sf, sf);
+        const __half2 s16h = __floats2half2_rn(sf * 0.0625f, sf * 0.0625f);
+        const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
+        const uint32_t s2_16 = *reinterpret_cast<const uint32_t*>(&s16h);
+        // codes landed (first K step of a copy), and the MMAs have released this A stage
+        const int sub = kb % CKB;
+        const bool got = (sub != 0 || mbar_wait_bounded(&c.code_full[cs], cphase, abort_flag, kTimeoutNs)) &&
+                         mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) fail(45);
+          ok = false;
+          break;
+        }
+        // row i of the copy: 128 bytes, 16-byte chunk k at position k ^ (i % 8)
+        const int chunk = sub * 2 + half;
+        const uint4 q = *reinterpret_cast<const uint4*>(smem_c + cs * C_BYTES + i * 128 + ((chunk ^ (i & 7)) << 4));
+        if (sub == CKB - 1 || kb == P.k_blocks - 1) {  // last K step of this copy
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.code_empty[cs]);
+          if (++cs == CSTAGES) {
+            cs = 0;
+            cphase ^= 1u;
+          }
+        }
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        unsigned char* dst = smem_a + stage * A_BYTES + i * 128;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = half * 4 + jj;  // 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4*>(dst + ((j ^ (i & 7)) << 4)) = dequant_word(qw[jj], s2, s2_16);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_peer(full_leader + static_cast<uint32_t>(stage * sizeof(uint64_t)));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------- epilogue (warps 0 .. 3) --
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t empty_leader = map_to_rank(smem_u32(&c.tmem_empty[0]), 0);
+    for (int t = pair; t < total_tiles; t += npairs) {
+      const Tile ti = decode(P, c, t);
+      const int N = P.n_out;
+      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
+      if (!named_barrier_and(1, 128, got)) {
+        if (lane == 0 && !got) fail(44);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * 256);
+      const int nch = ti.nmma / 32 + ((ti.nmma & 31) ? 1 : 0);
+      if (KIND == Kind::GateUp) {
+        // gate/up rows interleave as (b, u, r): a 16x256b load gives a thread
+        // the gate and the up value of one feature (as in the bf16 kernel)
+        const int f0 = ti.fidx * 128 + static_cast<int>(rank) * 64;
+        const float L = P.limit;
+        unsigned char* hb = reinterpret_cast<unsigned char*>(c.obuf);
+        __half* outh = static_cast<__half*>(P.out);
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          uint32_t v[2][16];
+          __syncwarp();
+          tmem_ld16x256b_x4(tbase + ch * 32, v[0]);
+          tmem_ld16x256b_x4(tbase + (16u << 16) + ch * 32, v[1]);
+          tmem_ld_wait();
+          named_barrier_sync(1, 128);  // previous chunk's staging reads done
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int fl = slot_of((2 * warp + h) * 8 + (lane >> 2));  // stored in the K order of the down MMA
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int tok = 8 * q + 2 * (lane & 3) + e;
+                const float gv = fminf(__uint_as_float(v[h][4 * q + e]), L);
+                const float uv = fminf(fmaxf(__uint_as_float(v[h][4 * q + 2 + e]), -L), L);
+                const float hv = __bfloat162float(__float2bfloat16_rn(__fdividef(gv, 1.f + __expf(-gv)) * uv));
+                *reinterpret_cast<__half*>(hb + tok * HPITCH + fl * 2) = __float2half_rn(hv);
+              }
+          }
+          named_barrier_sync(1, 128);  // staging complete
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int idx = threadIdx.x + 128 * r;
+            const int row = idx >> 3, c16 = idx & 7;
+            const int col = ch * 32 + row;
+            const int f = f0 + c16 * 8;
+            if (col < ti.ntok && f < N)
+              *reinterpret_cast<uint4*>(outh + static_cast<size_t>(ti.row0 + col) * N + f) =
+                  *reinterpret_cast<const uint4*>(hb + row * HPITCH + c16 * 16);
+          }
+        }
+      } else {
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(c.obuf);
+        __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(P.out);
+        const int nl = warp * 32 + lane;
+        const int n0 = ti.fidx * 256 + static_cast<int>(rank) * 128;
+        const float* rs = P.row_scale;
+#pragma unroll 1
+        for (int ch = 0; ch < nch; ++ch) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(tbase + ch * 32, v);
+          tmem_ld_wait();
+          const int mycol = ch * 32 + lane;
+          const float my_sc = (rs != nullptr && mycol < ti.ntok) ? rs[ti.row0 + mycol] : 1.f;
+          named_barrier_sync(1, 128);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float sc = __shfl_sync(0xffffffffu, my_sc, j);
+            ob[j * 128 + nl] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
+          }
+          named_barrier_sync(1, 128);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int idx = threadIdx.x + 128 * r;
+            const int row = idx >> 4, c16 = idx & 15;
+            const int col = ch * 32 + row;
+            const int n = n0 + c16 * 8;
+            if (col < ti.ntok && n < N)
+              *reinterpret_cast<uint4*>(outb + static_cast<size_t>(ti.row0 + col) * N + n) = c.obuf[idx];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(empty_leader + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the pair's MMAs, remote arrives and copies are done
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// Tokens for the gate/up MMA: fp16, each aligned 8 of K in the order
+// {0, 4, 1, 5, 2, 6, 3, 7}.  One thread per 8 values.
+__global__ void __launch_bounds__(256)
+    int4_tokens_prep_kernel(const __nv_bfloat16* __restrict__ x, long long n8, uint4* __restrict__ out) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n8) return;
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + idx);
+  const __half2 p0 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));  // x0, x4
+  const __half2 p1 = __floats2half2_rn(bf16hi(v.x), bf16hi(v.z));  // x1, x5
+  const __half2 p2 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));  // x2, x6
+  const __half2 p3 = __floats2half2_rn(bf16hi(v.y), bf16hi(v.w));  // x3, x7
+  uint4 o;
+  o.x = *reinterpret_cast<const uint32_t*>(&p0);
+  o.y = *reinterpret_cast<const uint32_t*>(&p1);
+  o.z = *reinterpret_cast<const uint32_t*>(&p2);
+  o.w = *reinterpret_cast<const uint32_t*>(&p3);
+  out[idx] = o;
+}
+
+bool encode_codes_gu(CUtensorMap* m, const void* q, int groups, int N, int K) {
+  // codes [G][2][N][K/2] bytes seen as {K/2, r = 8, u = 2, b = N/8, G}
+  const uint64_t row = static_cast<uint64_t>(K) / 2;
+  const uint64_t dims[5] = {row, 8, 2, static_cast<uint64_t>(N / 8), static_cast<uint64_t>(groups)};
+  const uint64_t strides[4] = {row, row * N, row * 8, row * N * 2};
+  const uint32_t box[5] = {CKB * BK / 2, 8, 2, 8, 1};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_codes_d(CUtensorMap* m, const void* q, int groups, int N, int K) {
+  const uint64_t row = static_cast<uint64_t>(K) / 2;
+  const uint64_t dims[3] = {row, static_cast<uint64_t>(N), static_cast<uint64_t>(groups)};
+  const uint64_t strides[2] = {row, row * N};
+  const uint32_t box[3] = {CKB * BK / 2, 128, 1};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool encode_tokens16(CUtensorMap* m, const void* base, int rows, int K) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {BK, TOK / 2};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <Kind KIND>
+int resident_pairs_int4() {
+  static int cached[64];
+  static bool known[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!known[dev]) {
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof(lc));
+    lc.gridDim = dim3(2);
+    lc.blockDim = dim3(THREADS);
+    lc.dynamicSmemBytes = kSmem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_int4_pair_kernel<KIND>, &lc) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cached[dev] = n;
+    known[dev] = true;
+  }
+  return cached[dev];
+}
+
+template <Kind KIND>
+cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offsets, int groups, const void* q,
+                             const void* scales, int N, int K, void* out, const float* row_scale, float limit,
+                             int32_t* err, int num_sms, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  Int4Params P;
+  memset(&P, 0, sizeof(P));
+  if (!encode_tokens16(&P.tma_x, tokens16, rows, K)) return cudaErrorInvalidValue;
+  const bool okq = KIND == Kind::GateUp ? encode_codes_gu(&P.tma_q, q, groups, N, K)
+                                        : encode_codes_d(&P.tma_q, q, groups, N, K);
+  if (!okq) return cudaErrorInvalidValue;
+  P.offsets = offsets;
+  P.scales = static_cast<const __nv_bfloat16*>(scales);
+  P.out = out;
+  P.row_scale = row_scale;
+  P.groups = groups;
+  P.rows = rows;
+  P.n_out = N;
+  P.K = K;
+  P.k_blocks = K / BK;
+  P.f_tiles = KIND == Kind::GateUp ? (N + 127) / 128 : (N + 255) / 256;
+  P.limit = limit;
+  P.err = err;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<KIND>), static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  int grid = std::max(2, num_sms / 2 * 2);
+  const int pairs = resident_pairs_int4<KIND>();
+  if (pairs > 0) grid = std::min(grid, 2 * pairs);
+  ffn_int4_pair_kernel<KIND><<<grid, THREADS, kSmem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool int4_prefill_preferred(int rows, int E) { return rows >= 32 * E; }
+
+cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
+                                    const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
+                                    void* y_perm, int32_t* err, int num_sms, cudaStream_t stream) {
+  const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
+  if (rows <= 0) return cudaSuccess;
+  const long long n8 = static_cast<long long>(rows) * (H / 8);
+  int4_tokens_prep_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x_perm), n8, static_cast<uint4*>(tokens16));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_int4_pair<Kind::GateUp>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, I, H, h16, nullptr,
+                                     cfg.swiglu_limit, err, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  return launch_int4_pair<Kind::Down>(h16, rows, offsets, E, w.w_down, w.s_down, H, I, y_perm, w_perm, 0.f, err,
+                                      num_sms, stream);
+}
+
+}  // namespace moe

@@ -122,13 +122,20 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
     MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
     MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, sms, stream));
   } else {
-    // gate/up in fp32 into the h region; the SwiGLU is applied while the
-    // down projection's activations are prepared
     void* act16 = at<void>(ws, L.act16);
-    float* gu = at<float>(ws, L.h);
-    MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, stream));
-    if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, stream));
+    if (int4_prefill_preferred(R, E)) {
+      // many tokens per expert: dequantise in shared memory, tensor cores
+      MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_perm, offsets, R, act16, at<void>(ws, L.h), w_perm, y_perm,
+                                           err, sms, stream));
+      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+    } else {
+      // gate/up in fp32 into the h region; the SwiGLU is applied while the
+      // down projection's activations are prepared
+      float* gu = at<float>(ws, L.h);
+      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, stream));
+      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+      MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, stream));
+    }
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
   }
   return MOE_OK;

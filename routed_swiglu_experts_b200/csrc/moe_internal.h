@@ -82,6 +82,14 @@ cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, con
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
                               int rows, void* act16, const float* w_perm, void* y_perm, cudaStream_t stream);
 
+// W4A16 grouped GEMMs for many tokens per expert: int4 codes dequantised to
+// fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.
+// tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16.
+bool int4_prefill_preferred(int rows, int E);
+cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
+                                    const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
+                                    void* y_perm, int32_t* err, int num_sms, cudaStream_t stream);
+
 // Shared expert for T <= 32 tokens: split-K tensor-core GEMMs streaming the
 // weights across all SMs, then an ordered sum of the K slices.
 constexpr int kDenseSmallMaxTokens = 32;

@@ -46,6 +46,13 @@ EDGE = {
     "w4a16_small": LayerConfig("w4a16_small", T=20, H=256, E=6, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
                                bias_range=0.05, w4a16=True),
     "w4a16_many_tokens": LayerConfig("w4a16_many_tokens", T=96, H=384, E=3, k=2, I=256, I_s=0, w4a16=True),
+    # fewer than 32 rows per expert on average: the GEMV path, several 8-token chunks per expert
+    "w4a16_chunks": LayerConfig("w4a16_chunks", T=40, H=256, E=8, k=2, I=128, I_s=0, w4a16=True),
+    # 32 rows per expert or more: the grouped prefill GEMM (int4 dequantised in shared memory)
+    "w4a16_prefill": LayerConfig("w4a16_prefill", T=700, H=512, E=8, k=2, I=384, I_s=256, alpha=2.5, renorm=True,
+                                 bias_range=0.05, w4a16=True),
+    "w4a16_prefill_clamp": LayerConfig("w4a16_prefill_clamp", T=300, H=256, E=4, k=2, I=256, I_s=128,
+                                       swiglu_limit=0.5, w4a16=True),
     "shared_small_t32": LayerConfig("shared_small_t32", T=32, H=256, E=4, k=2, I=64, I_s=96, alpha=2.5,
                                     renorm=True),
     "shared_tc_t33": LayerConfig("shared_tc_t33", T=33, H=256, E=4, k=2, I=64, I_s=96),
@@ -151,8 +158,8 @@ def test_tied_router_prefers_lower_id(small_inputs):
 
 # ------------------------------------------------------ benchmark layers ----
 
-FULL = ["mid", "skewed", "large_prefill", "decode_w4a16"]
-SAMPLE_TOKENS = {"mid": 96, "skewed": 64, "large_prefill": 12, "decode_w4a16": 12}
+FULL = ["mid", "skewed", "large_prefill", "decode_w4a16", "prefill_w4a16"]
+SAMPLE_TOKENS = {"mid": 96, "skewed": 64, "large_prefill": 12, "decode_w4a16": 12, "prefill_w4a16": 12}
 
 
 @pytest.mark.parametrize("name", FULL)
