@@ -221,6 +221,33 @@ def base_line(args, n_gpus, cfg):
     }
 
 
+# ------------------------------------------------------- replicas (N > 1) ----
+
+def rank_barrier(world):
+    """Barrier over the job's ranks (no-op for one rank)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_max(v, world, device):
+    """Max of a per-rank float over the job's ranks: every timed figure is
+    the slowest rank's."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(world, tokens_per_rank, ms_per_step):
+    """Whole-job throughput of N replicas: every rank processes its own
+    tokens each step; the step time is the max over ranks."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # --------------------------------------------------------------- our arm ----
 
 def bench_ours(args, rank, world, local_rank):
@@ -248,15 +275,10 @@ def bench_ours(args, rank, world, local_rank):
     clocks = ClockSampler(gpu_uuid(dev))
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(v, world, dev)
 
     for _ in range(args.warmup):
         layer.forward(x, out=out)
@@ -377,7 +399,7 @@ def bench_ours(args, rank, world, local_rank):
                 "routed_tflops": routed_f / ffn_s / 1e12}
     line = base_line(args, world, c)
     line.update({
-        "value": world * c.T / (ms_per_step / 1e3), "ms_per_step": ms_per_step, "dtype": "bf16",
+        "value": replica_tokens_per_s(world, c.T, ms_per_step), "ms_per_step": ms_per_step, "dtype": "bf16",
         "roofline": roof,
         "stage_ms": stage_ms,
         "e2e": {"value": world * c.T / (e2e_ms / 1e3), "unit": "tokens/s",
