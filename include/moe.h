@@ -166,9 +166,12 @@ MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids,
  *   y_perm[r] = bf16( w_perm[r] * W_down[e] h ),
  *   h = bf16( silu(min(W_gate[e] x_perm[r], L)) * clamp(W_up[e] x_perm[r], -L, L) )
  * ([glm5next] §Numerics: asymmetric clamp).  w_perm == NULL: unweighted.
- * bf16 weights run on the tcgen05 tensor cores; MOE_W_INT4_G128 weights run
- * the W4A16 kernels that dequantise in registers ([glm5next]
- * W4A16_GEMV_MODULE).
+ * bf16 weights run on the tcgen05 tensor cores.  MOE_W_INT4_G128 weights
+ * run the W4A16 GEMV kernels that dequantise in registers ([glm5next]
+ * W4A16_GEMV_MODULE) when there are fewer than 32 routed rows per expert on
+ * average, else a grouped tensor-core GEMM that dequantises the int4 codes
+ * into fp16 tiles in shared memory ([glm5next] MOE_GROUPED_MODULE); both
+ * round h to bf16 as the bf16 path does.
  * When x_shared != NULL the shared expert runs in the same launches:
  *   shared_out[t] = bf16( SwiGLU_clamped FFN_shared(x_shared[t]) ), unscaled.
  *   x_perm          bf16 [T*k, H]    expert_offsets int32 [E+1]
