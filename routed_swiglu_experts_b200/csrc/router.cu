@@ -1,5 +1,5 @@
-// Router: the fp32 logits GEMM runs on the tensor cores (grouped_gemm.cu,
-// router mode) on an exact bf16 split of the fp32 weight; here are the split
+// Router: the fp32 logits GEMM runs on the tensor cores (splitk_gemm.cu, three
+// passes over K) on an exact bf16 split of the fp32 weight; here are the split
 // and the warp-per-token sigmoid + biased top-k with an fp64 re-rank of
 // near-ties.
 //

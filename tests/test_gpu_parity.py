@@ -146,6 +146,32 @@ def test_forward_is_deterministic(small_inputs):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("name", ["ragged", "w4a16_small", "w4a16_prefill", "shared_small_t32"])
+def test_forward_replays_from_a_cuda_graph(small_inputs, name):
+    """The forward enqueues only device work on the given stream (no host
+    sync, no allocation): captured once into a CUDA graph, its replay gives
+    the eager forward's bits, also on a non-default stream."""
+    inp = small_inputs[name]
+    layer = gpu_layer(inp)
+    x = inp.x.cuda()
+    eager = layer.forward(x).clone()
+    side = torch.cuda.Stream()
+    out = torch.empty_like(eager)
+    with torch.cuda.stream(side):
+        layer.forward(x, out=out, stream=side)   # warm: every one-time setup happens here
+    side.synchronize()
+    assert torch.equal(out, eager)
+    out.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        layer.forward(x, out=out, stream=side)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    assert layer.device_error() == 0
+    del graph
+
+
 def test_tied_router_prefers_lower_id(small_inputs):
     inp = small_inputs["tied_router"]
     layer = gpu_layer(inp)
