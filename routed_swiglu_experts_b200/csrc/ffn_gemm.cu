@@ -21,6 +21,13 @@
 // Roles per CTA (192 threads): warps 0-3 epilogue (TMEM -> registers ->
 // global), warp 4 TMA producer, warp 5 TMEM owner (+ MMA issuer in the first
 // CTA).  6-stage ring of 32 KB; two 256-column fp32 accumulators per CTA.
+// Persistent: one pair per two SMs takes tiles from a queue (an atomic
+// counter in the workspace header) in the fixed tile order below, so the
+// pairs that draw ragged last tiles take more of them; a fixed round-robin
+// split of the same order left whole pairs with only full tiles (an even
+// pair count against an even tile count per expert).  The first CTA's
+// producer takes each id and hands it to every role of both CTAs through a
+// small ring of ids guarded by mbarriers.
 // gate/up weight rows of a CTA cover 64 features, loaded through a 5-D view of
 // the [gate; up] weight so that shared-memory row 16b + 8u + r is the gate
 // (u = 0) or up (u = 1) row of feature 8b + r.  A 16-lane TMEM load then hands
@@ -46,6 +53,10 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr int HPITCH = 144;                // bytes per token row of the staged gate/up output (64 bf16 + pad)
+constexpr int QD = 8;                      // tile-id ring depth
+// readers of every tile id: the MMA issuer and 4 epilogue warps of the first
+// CTA, the TMA producer and 4 epilogue warps of the second
+constexpr uint32_t kTileReaders = 1 + 4 + 1 + 4;
 
 enum class Kind { GateUp, Down };
 
@@ -63,6 +74,7 @@ struct alignas(64) PairParams {
   int32_t nprob;
   float limit;
   int32_t* err;
+  int32_t* queue;             // {next tile, pairs retired}: zero at launch, left zero at exit
 };
 
 struct Ctl {
@@ -71,6 +83,9 @@ struct Ctl {
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t mma_done;
+  uint64_t tq_full[QD];             // tile id published (one arrive)
+  uint64_t tq_empty[QD];            // first CTA: every reader has taken it
+  int32_t tq[QD];                   // tile ids; -1 = no more tiles
   uint32_t tmem_base;
   int32_t abort_flag;
   int32_t tiles[2];
@@ -87,8 +102,9 @@ struct Tile {
 };
 
 // Tile order: problem 0 then 1; group by group; inside a group weight-row
-// tile major, token tile minor (the token tiles of one weight slice run back
-// to back and share it through L2).
+// tile major, token tile minor (the token tiles of one weight slice are
+// handed out back to back, run at the same time on neighbouring pairs and
+// share it through L2).
 __device__ __forceinline__ Tile decode(const PairParams& P, const Ctl& c, int t) {
   Tile ti;
   ti.p = 0;
@@ -140,7 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -152,6 +168,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&c.tmem_empty[a], 2 * 4);
     }
     mbar_init(&c.mma_done, 1);
+    for (int i = 0; i < QD; ++i) {
+      mbar_init(&c.tq_full[i], 1);
+      mbar_init(&c.tq_empty[i], kTileReaders);
+    }
     c.abort_flag = 0;
     fence_mbar_init();
   }
@@ -224,10 +244,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      int t_next = -2;  // next queue position, once fetched
+      for (;;) {
+        // Next tile: the first CTA takes it from the launch's queue and
+        // publishes it to both CTAs; tiles go out in order to whichever pair
+        // asks first, so pairs that drew cheap (ragged) tiles take more.
+        int t;
+        if (leader) {
+          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, kTimeoutNs)) {
+            fail(35);
+            break;
+          }
+          if (t_next == -2) t_next = atomicAdd(P.queue, 1);
+          t = t_next < total_tiles ? t_next : -1;
+          t_next = -2;
+          c.tq[q] = t;
+          st_cluster_u32(map_to_rank(smem_u32(&c.tq[q]), 1), static_cast<uint32_t>(t));
+          mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
+          mbar_arrive(&c.tq_full[q]);
+        } else {
+          if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, kTimeoutNs)) {
+            fail(36);
+            break;
+          }
+          t = c.tq[q];
+          mbar_arrive_cluster(leader_bar(&c.tq_empty[q]));
+        }
+        if (++q == QD) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const int p = ti.p;
         const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
+        // the next id is fetched a few stages before this tile's last copy,
+        // so the atomic's round trip overlaps the copies
+        const int kpre = P.k_blocks[p] > 3 ? P.k_blocks[p] - 3 : 0;
         for (int kb = 0; kb < P.k_blocks[p]; ++kb) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             fail(31);
@@ -246,11 +301,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
           }
           tma_load_2d_pair(smem_b + stage * B_BYTES, &P.tma_x[p], kc, xrow, bar);
+          if (leader && kb == kpre) t_next = atomicAdd(P.queue, 1);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+        }
+        if (!ok) break;
+      }
+      if (leader) {
+        // retire from the queue; the last pair of the launch resets it (every
+        // pair has taken its final tile id before it retires)
+        __threadfence();
+        if (atomicAdd(P.queue + 1, 1) == npairs - 1) {
+          __threadfence();
+          atomicExch(P.queue, 0);
+          atomicExch(P.queue + 1, 0);
         }
       }
       if (leader) {  // drain: the last copy of each stage (both CTAs' bytes land here)
@@ -269,7 +336,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      for (;;) {
+        if (!mbar_wait_bounded(&c.tq_full[q], qph, abort_flag, kTimeoutNs)) {
+          fail(37);
+          break;
+        }
+        const int t = c.tq[q];
+        mbar_arrive(&c.tq_empty[q]);
+        if (++q == QD) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const int p = ti.p;
         const uint32_t idesc = umma_idesc_bf16(2 * ROWS, ti.nmma);
@@ -315,7 +395,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t acc_phase = 0;
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t empty_leader = map_to_rank(smem_u32(&c.tmem_empty[0]), 0);
-    for (int t = pair; t < total_tiles; t += npairs) {
+    const uint32_t tq_empty_leader = map_to_rank(smem_u32(&c.tq_empty[0]), 0);
+    int q = 0;
+    uint32_t qph = 0;
+    for (;;) {
+      const bool gotq = mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, kTimeoutNs);
+      if (!named_barrier_and(1, 128, gotq)) {
+        if (lane == 0 && !gotq) fail(40);
+        break;
+      }
+      const int t = c.tq[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tq_empty_leader + static_cast<uint32_t>(q * sizeof(uint64_t)));
+      if (++q == QD) {
+        q = 0;
+        qph ^= 1u;
+      }
+      if (t < 0) break;
       const Tile ti = decode(P, c, t);
       const int p = ti.p;
       const int N = P.n_out[p];
@@ -474,8 +570,8 @@ int resident_pairs() {
 }
 
 template <Kind KIND>
-cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err, int num_sms,
-                        cudaStream_t stream) {
+cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
+                        int32_t* queue, int num_sms, cudaStream_t stream) {
   PairParams P;
   memset(&P, 0, sizeof(P));
   const FfnProblem* probs[2];
@@ -500,9 +596,11 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
     P.k_blocks[i] = (f.K + BK - 1) / BK;
     P.f_tiles[i] = KIND == Kind::GateUp ? (f.N + 127) / 128 : (f.N + 255) / 256;
   }
+  if (queue == nullptr) return cudaErrorInvalidValue;
   P.nprob = np;
   P.limit = limit;
   P.err = err;
+  P.queue = queue;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<KIND>), static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   int grid = std::max(2, num_sms / 2 * 2);
@@ -515,13 +613,13 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
 }  // namespace
 
 cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
-                               int num_sms, cudaStream_t stream) {
-  return launch_pair<Kind::GateUp>(routed, shared, limit, err, num_sms, stream);
+                               int32_t* queue, int num_sms, cudaStream_t stream) {
+  return launch_pair<Kind::GateUp>(routed, shared, limit, err, queue, num_sms, stream);
 }
 
-cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int num_sms,
-                             cudaStream_t stream) {
-  return launch_pair<Kind::Down>(routed, shared, 0.f, err, num_sms, stream);
+cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int32_t* queue,
+                             int num_sms, cudaStream_t stream) {
+  return launch_pair<Kind::Down>(routed, shared, 0.f, err, queue, num_sms, stream);
 }
 
 }  // namespace moe

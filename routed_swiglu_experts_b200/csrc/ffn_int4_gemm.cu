@@ -19,7 +19,8 @@
 // weights sit in the order {0, 4, 1, 5, 2, 6, 3, 7} (how four LOP3s split a
 // 32-bit code word); the tokens are prepared in the same order, and the
 // gate/up epilogue writes h in it, so the K sum is unchanged.
-// Every mbarrier wait is bounded (MOE_ERR_DEVICE_TIMEOUT on expiry).
+// Tiles are handed out from a queue in the workspace header as in the bf16
+// kernel.  Every mbarrier wait is bounded (MOE_ERR_DEVICE_TIMEOUT on expiry).
 #include <cstring>
 
 #include <cuda_fp16.h>
@@ -45,6 +46,10 @@ constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;  // 0-3 epilogue, 4 token TM
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr int HPITCH = 144;                  // bytes per token row of the staged gate/up output
+constexpr int QD = 8;                        // tile-id ring depth
+// readers of every tile id, per CTA: token TMA (second CTA) or MMA issuer
+// (first CTA), code TMA, 8 dequantisation warps, 4 epilogue warps
+constexpr uint32_t kTileReaders = 2 * (1 + 1 + DQ_WARPS + 4);
 
 enum class Kind { GateUp, Down };
 
@@ -63,6 +68,7 @@ struct alignas(64) Int4Params {
   int32_t f_tiles;
   float limit;
   int32_t* err;
+  int32_t* queue;             // {next tile, pairs retired}: zero at launch, left zero at exit
 };
 
 struct Ctl {
@@ -74,6 +80,9 @@ struct Ctl {
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t mma_done;
+  uint64_t tq_full[QD];       // tile id published (one arrive)
+  uint64_t tq_empty[QD];      // first CTA: every reader has taken it
+  int32_t tq[QD];             // tile ids; -1 = no more tiles
   uint32_t tmem_base;
   int32_t abort_flag;
   int32_t tiles;
@@ -136,6 +145,21 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
   return r;
 }
 
+// Reader side of the tile-id ring: wait until slot q holds the next id (it
+// may have been stored by the other CTA of the pair: cluster-scope acquire).
+__device__ __forceinline__ bool wait_tile(Ctl& c, int q, uint32_t qph, volatile int32_t* abort, int& t) {
+  if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort, kTimeoutNs)) return false;
+  t = c.tq[q];
+  return true;
+}
+__device__ __forceinline__ void release_tile(Ctl& c, int q) { mbar_arrive_cluster(leader_bar(&c.tq_empty[q])); }
+__device__ __forceinline__ void next_slot(int& q, uint32_t& qph) {
+  if (++q == QD) {
+    q = 0;
+    qph ^= 1u;
+  }
+}
+
 // Position of feature f inside its aligned 8 after the {0,4,1,5,2,6,3,7} order.
 __device__ __forceinline__ int slot_of(int f) {
   const int j = f & 7;
@@ -156,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -173,6 +197,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&c.tmem_empty[a], 2 * 4);
     }
     mbar_init(&c.mma_done, 1);
+    for (int i = 0; i < QD; ++i) {
+      mbar_init(&c.tq_full[i], 1);
+      mbar_init(&c.tq_empty[i], kTileReaders);
+    }
     c.abort_flag = 0;
     fence_mbar_init();
   }
@@ -233,9 +261,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      int t_next = -2;  // next queue position, once fetched
+      for (;;) {
+        // Next tile: this thread of the first CTA takes it from the launch's
+        // queue and publishes it to every role of both CTAs.
+        int t;
+        if (leader) {
+          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, kTimeoutNs)) {
+            fail(50);
+            break;
+          }
+          if (t_next == -2) t_next = atomicAdd(P.queue, 1);
+          t = t_next < total_tiles ? t_next : -1;
+          t_next = -2;
+          c.tq[q] = t;
+          st_cluster_u32(map_to_rank(smem_u32(&c.tq[q]), 1), static_cast<uint32_t>(t));
+          mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
+          mbar_arrive(&c.tq_full[q]);
+        } else {
+          if (!wait_tile(c, q, qph, abort_flag, t)) {
+            fail(51);
+            break;
+          }
+          release_tile(c, q);
+        }
+        next_slot(q, qph);
+        if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
+        const int kpre = P.k_blocks > 3 ? P.k_blocks - 3 : 0;  // fetch the next id a few copies early
         for (int kb = 0; kb < P.k_blocks; ++kb) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             fail(41);
@@ -244,11 +300,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           if (leader) mbar_arrive_expect_tx(&c.tok_full[stage], 2 * B_BYTES);
           tma_load_2d_pair(smem_b + stage * B_BYTES, &P.tma_x, kb * BK, xrow, leader_bar(&c.tok_full[stage]));
+          if (leader && kb == kpre) t_next = atomicAdd(P.queue, 1);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+        }
+        if (!ok) break;
+      }
+      if (leader) {
+        // retire from the queue; the last pair of the launch resets it
+        __threadfence();
+        if (atomicAdd(P.queue + 1, 1) == npairs - 1) {
+          __threadfence();
+          atomicExch(P.queue, 0);
+          atomicExch(P.queue + 1, 0);
         }
       }
       // drain (first CTA): the last token copies of both CTAs complete on
@@ -268,7 +335,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      for (;;) {
+        int t;
+        if (!wait_tile(c, q, qph, abort_flag, t)) {
+          fail(52);
+          break;
+        }
+        release_tile(c, q);
+        next_slot(q, qph);
+        if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const uint32_t idesc = umma_idesc_f16(2 * ROWS, ti.nmma);
         if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
@@ -315,7 +392,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t cphase = 0;
       bool ok = true;
       const int ncb = (P.k_blocks + CKB - 1) / CKB;
-      for (int t = pair; t < total_tiles && ok; t += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      for (;;) {
+        int t;
+        if (!wait_tile(c, q, qph, abort_flag, t)) {
+          fail(53);
+          break;
+        }
+        release_tile(c, q);
+        next_slot(q, qph);
+        if (t < 0) break;
         const Tile ti = decode(P, c, t);
         for (int cb = 0; cb < ncb; ++cb) {
           if (!mbar_wait_bounded(&c.code_empty[cs], cphase ^ 1u, abort_flag, kTimeoutNs)) {
@@ -338,6 +425,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             cphase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       // drain: the last code copy of each stage
       const int nst = issued < CSTAGES ? issued : CSTAGES;
@@ -359,7 +447,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t full_leader = leader_bar(&c.full[0]);
     int stage = 0, cs = 0;
     uint32_t phase = 0, cphase = 0;
-    for (int t = pair; t < total_tiles; t += npairs) {
+    int q = 0;
+    uint32_t qph = 0;
+    for (;;) {
+      int t = -1;
+      const bool gotq = wait_tile(c, q, qph, abort_flag, t);
+      if (!__all_sync(0xffffffffu, gotq)) {
+        if (lane == 0) fail(54);
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) release_tile(c, q);
+      next_slot(q, qph);
+      if (t < 0) break;
       const Tile ti = decode(P, c, t);
       // this row's scales (nullptr: past the end of the matrix, codes are zero-filled)
       const __nv_bfloat16* sp = nullptr;
@@ -441,7 +541,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t acc_phase = 0;
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t empty_leader = map_to_rank(smem_u32(&c.tmem_empty[0]), 0);
-    for (int t = pair; t < total_tiles; t += npairs) {
+    int q = 0;
+    uint32_t qph = 0;
+    for (;;) {
+      int t = -1;
+      const bool gotq = wait_tile(c, q, qph, abort_flag, t);
+      if (!named_barrier_and(1, 128, gotq)) {
+        if (lane == 0 && !gotq) fail(55);
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) release_tile(c, q);
+      next_slot(q, qph);
+      if (t < 0) break;
       const Tile ti = decode(P, c, t);
       const int N = P.n_out;
       const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
@@ -614,8 +726,9 @@ int resident_pairs_int4() {
 template <Kind KIND>
 cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offsets, int groups, const void* q,
                              const void* scales, int N, int K, void* out, const float* row_scale, float limit,
-                             int32_t* err, int num_sms, cudaStream_t stream) {
+                             int32_t* err, int32_t* queue, int num_sms, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
+  if (queue == nullptr) return cudaErrorInvalidValue;
   Int4Params P;
   memset(&P, 0, sizeof(P));
   if (!encode_tokens16(&P.tma_x, tokens16, rows, K)) return cudaErrorInvalidValue;
@@ -634,6 +747,7 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
   P.f_tiles = KIND == Kind::GateUp ? (N + 127) / 128 : (N + 255) / 256;
   P.limit = limit;
   P.err = err;
+  P.queue = queue;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<KIND>), static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   int grid = std::max(2, num_sms / 2 * 2);
@@ -649,7 +763,7 @@ bool int4_prefill_preferred(int rows, int E) { return rows >= 32 * E; }
 
 cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
                                     const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
-                                    void* y_perm, int32_t* err, int num_sms, cudaStream_t stream) {
+                                    void* y_perm, int32_t* err, int32_t* queues, int num_sms, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
   if (rows <= 0) return cudaSuccess;
   const long long n8 = static_cast<long long>(rows) * (H / 8);
@@ -658,10 +772,10 @@ cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_int4_pair<Kind::GateUp>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, I, H, h16, nullptr,
-                                     cfg.swiglu_limit, err, num_sms, stream);
+                                     cfg.swiglu_limit, err, queues, num_sms, stream);
   if (e != cudaSuccess) return e;
   return launch_int4_pair<Kind::Down>(h16, rows, offsets, E, w.w_down, w.s_down, H, I, y_perm, w_perm, 0.f, err,
-                                      num_sms, stream);
+                                      queues + 2, num_sms, stream);
 }
 
 }  // namespace moe

@@ -52,6 +52,7 @@ T* at(void* ws, size_t off) {
 }
 
 int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
+int32_t* tile_queue(void* ws, TileQueueSlot slot) { return reinterpret_cast<WsHeader*>(ws)->tile_queue + slot; }
 
 bool is_int4(const moe_config& cfg) { return cfg.expert_format == MOE_W_INT4_G128; }
 
@@ -99,6 +100,8 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   const int H = cfg.hidden, I = cfg.expert_inter, Is = cfg.shared_inter, E = cfg.num_experts;
   const int R = T * cfg.top_k;
   int32_t* err = err_word(ws);
+  int32_t* qgu = tile_queue(ws, kQueueGateUp);
+  int32_t* qd = tile_queue(ws, kQueueDown);
   void* h = at<void>(ws, L.h);
   void* hs = at<void>(ws, L.h_shared);
   const int sms = num_sms_current_device();
@@ -119,24 +122,24 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   if (!is_int4(cfg)) {
     FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
-    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, sms, stream));
-    MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, qgu, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, qd, sms, stream));
   } else {
     void* act16 = at<void>(ws, L.act16);
     if (int4_prefill_preferred(R, E)) {
       // many tokens per expert: dequantise in shared memory, tensor cores
       MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_perm, offsets, R, act16, at<void>(ws, L.h), w_perm, y_perm,
-                                           err, sms, stream));
-      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+                                           err, tile_queue(ws, kQueueInt4GateUp), sms, stream));
+      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
     } else {
       // gate/up in fp32 into the h region; the SwiGLU is applied while the
       // down projection's activations are prepared
       float* gu = at<float>(ws, L.h);
       MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, stream));
-      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, sms, stream));
+      if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
       MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, stream));
     }
-    if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, sms, stream));
+    if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, qd, sms, stream));
   }
   return MOE_OK;
 }

@@ -16,9 +16,14 @@ namespace moe {
 struct WsHeader {
   int32_t error;       // first device error (MOE_ERR_DEVICE_TIMEOUT ...)
   int32_t detail;      // which wait gave up (kernel-specific code)
-  int32_t pad[62];
+  // Tile queues of the persistent grouped GEMMs, {next tile, pairs retired}
+  // per kernel: zero when a launch starts, reset to zero by the last CTA
+  // pair of every launch.
+  int32_t tile_queue[8];
+  int32_t pad[54];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+enum TileQueueSlot { kQueueGateUp = 0, kQueueDown = 2, kQueueInt4GateUp = 4, kQueueInt4Down = 6 };
 
 __device__ __forceinline__ void report_error(int32_t* err, int32_t code, int32_t detail) {
   if (err != nullptr && atomicCAS(err, 0, code) == 0) err[1] = detail;
@@ -61,27 +66,41 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// kCluster: acquire at cluster scope, for data that a thread of the other
+// CTA of the pair stored into this CTA's shared memory before its
+// release.cluster arrive.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
+  if (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 
 // Bounded wait on phase `parity` of `bar`.  Gives up when `abort` becomes
 // non-zero or after `limit_ns` nanoseconds; returns false in that case.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int32_t* abort, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  if (mbar_try_wait<kCluster>(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait<kCluster>(a, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
@@ -168,6 +187,11 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 // loads of the other CTA.
 __device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 32-bit store into the shared memory of a CTA of the cluster.
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // shared::cluster address of the mbarrier at the same offset as `bar` in the

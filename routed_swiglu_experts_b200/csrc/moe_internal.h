@@ -70,10 +70,11 @@ struct FfnProblem {
   void* out;                     // bf16 [rows, N]
   const float* row_scale;        // per-row scale (down only) or nullptr
 };
+// queue: the launch's two tile-queue words in the workspace header (zero).
 cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
-                               int num_sms, cudaStream_t stream);
-cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int num_sms,
-                             cudaStream_t stream);
+                               int32_t* queue, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int32_t* queue,
+                             int num_sms, cudaStream_t stream);
 
 // W4A16 routed expert kernels (dequantise in registers).
 // act16: scratch for the activations in MMA slot order (fp16, [rows, K]).
@@ -84,11 +85,12 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
 
 // W4A16 grouped GEMMs for many tokens per expert: int4 codes dequantised to
 // fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.
-// tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16.
+// tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16; queues:
+// four tile-queue words in the workspace header (gate/up, then down).
 bool int4_prefill_preferred(int rows, int E);
 cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
                                     const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
-                                    void* y_perm, int32_t* err, int num_sms, cudaStream_t stream);
+                                    void* y_perm, int32_t* err, int32_t* queues, int num_sms, cudaStream_t stream);
 
 // Shared expert for T <= 32 tokens: split-K tensor-core GEMMs streaming the
 // weights across all SMs, then an ordered sum of the K slices.

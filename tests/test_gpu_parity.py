@@ -146,6 +146,24 @@ def test_forward_is_deterministic(small_inputs):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("name", ["ragged", "w4a16_prefill"])
+def test_tile_queues_are_left_at_zero(small_inputs, name):
+    """The persistent grouped GEMMs hand tiles out from counters in the
+    workspace header; every launch must leave them at zero, so that the next
+    call on the same workspace (or a graph replay) starts from tile 0."""
+    inp = small_inputs[name]
+    layer = gpu_layer(inp)
+    x = inp.x.cuda()
+    outs = []
+    for _ in range(3):
+        outs.append(layer.forward(x).clone())
+        torch.cuda.synchronize()
+        header = layer.ws[:256].view(torch.int32).cpu()
+        assert header[0].item() == 0, "device error word set"
+        assert torch.count_nonzero(header[2:10]).item() == 0, f"tile queue words {header[2:10].tolist()}"
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
 @pytest.mark.parametrize("name", ["ragged", "w4a16_small", "w4a16_prefill", "shared_small_t32"])
 def test_forward_replays_from_a_cuda_graph(small_inputs, name):
     """The forward enqueues only device work on the given stream (no host
