@@ -122,8 +122,9 @@ MOE_API moe_status moe_config_validate(const moe_config* cfg);
  * to `max_tokens` tokens.  *bytes is written on MOE_OK. */
 MOE_API moe_status moe_workspace_size(const moe_config* cfg, int32_t max_tokens, size_t* bytes);
 
-/* Zero the workspace header (device error word) on `stream`.  Call once
- * after allocating a workspace. */
+/* Zero the workspace header on `stream`: the device error word and the
+ * tile counters of the grouped GEMMs (every launch leaves those at zero
+ * again).  Call once after allocating a workspace. */
 MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Router: logit[t, e] = sum_h x[t, h] * router_w[e, h] in fp32 ([beam]
