@@ -20,7 +20,11 @@
 //
 // Roles per CTA (192 threads): warps 0-3 epilogue (TMEM -> registers ->
 // global), warp 4 TMA producer, warp 5 TMEM owner (+ MMA issuer in the first
-// CTA).  6-stage ring of 32 KB; two 256-column fp32 accumulators per CTA.
+// CTA).  3-stage ring of 64 KB, each stage two 64-deep K chunks of weights
+// and tokens (one barrier round trip and one commit per 128 of K: the
+// per-step handshake, not the bytes, is what a tile pays whatever its token
+// count; 6 stages of 32 KB ran 2-4% slower); two 256-column fp32
+// accumulators per CTA.
 // Persistent: one pair per two SMs takes tiles from a queue (an atomic
 // counter in the workspace header) in the fixed tile order below, so the
 // pairs that draw ragged last tiles take more of them; a fixed round-robin
@@ -45,10 +49,13 @@ namespace {
 constexpr int BK = 64;
 constexpr int ROWS = 128;                  // weight rows per CTA (A half)
 constexpr int TOK = 256;                   // tokens per pair tile (MMA N <= 256)
-constexpr int STAGES = 6;
-constexpr int A_BYTES = ROWS * BK * 2;     // 16 KB
-constexpr int B_BYTES = (TOK / 2) * BK * 2;  // 16 KB: this CTA's half of the tokens
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int KCH = 2;                     // 64-deep K chunks per pipeline stage
+constexpr int STAGES = 6 / KCH;
+constexpr int A_BYTES = ROWS * BK * 2;     // 16 KB per chunk
+constexpr int B_BYTES = (TOK / 2) * BK * 2;  // 16 KB per chunk: this CTA's half of the tokens
+constexpr int A_STAGE = KCH * A_BYTES;
+constexpr int B_STAGE = KCH * B_BYTES;
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -150,7 +157,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
   unsigned char* smem_a = smem;
-  unsigned char* smem_b = smem + STAGES * A_BYTES;
+  unsigned char* smem_b = smem + STAGES * A_STAGE;
   Ctl& c = *reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -282,26 +289,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
         // the next id is fetched a few stages before this tile's last copy,
         // so the atomic's round trip overlaps the copies
-        const int kpre = P.k_blocks[p] > 3 ? P.k_blocks[p] - 3 : 0;
-        for (int kb = 0; kb < P.k_blocks[p]; ++kb) {
+        const int nkb = P.k_blocks[p];
+        const int nstage = (nkb + KCH - 1) / KCH;  // the last stage of an odd count holds one chunk
+        const int kpre = nstage > 2 ? nstage - 2 : 0;
+        for (int st = 0; st < nstage; ++st) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             fail(31);
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&c.full[stage], 2 * STAGE_BYTES);
+          const int nk = min(KCH, nkb - st * KCH);
+          if (leader) mbar_arrive_expect_tx(&c.full[stage], 2u * static_cast<uint32_t>(nk * (A_BYTES + B_BYTES)));
           const uint32_t bar = leader_bar(&c.full[stage]);
-          const int kc = kb * BK;
-          unsigned char* sa = smem_a + stage * A_BYTES;
-          if (KIND == Kind::GateUp) {
-            const int fb = ti.fidx * 16 + static_cast<int>(rank) * 8;  // first 8-feature block
-            tma_load_5d_pair(sa, &P.tma_w[p], kc, 0, 0, fb, ti.g, bar);
-          } else {
-            const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
-            tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
+          for (int ch = 0; ch < nk; ++ch) {
+            const int kc = (st * KCH + ch) * BK;
+            unsigned char* sa = smem_a + stage * A_STAGE + ch * A_BYTES;  // 1024-byte aligned
+            if (KIND == Kind::GateUp) {
+              const int fb = ti.fidx * 16 + static_cast<int>(rank) * 8;  // first 8-feature block
+              tma_load_5d_pair(sa, &P.tma_w[p], kc, 0, 0, fb, ti.g, bar);
+            } else {
+              const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
+              tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
+            }
+            tma_load_2d_pair(smem_b + stage * B_STAGE + ch * B_BYTES, &P.tma_x[p], kc, xrow, bar);
           }
-          tma_load_2d_pair(smem_b + stage * B_BYTES, &P.tma_x[p], kc, xrow, bar);
-          if (leader && kb == kpre) t_next = atomicAdd(P.queue, 1);
+          if (leader && st == kpre) t_next = atomicAdd(P.queue, 1);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -359,19 +371,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-        for (int kb = 0; kb < P.k_blocks[p]; ++kb) {
+        const int nkb = P.k_blocks[p];
+        const int nstage = (nkb + KCH - 1) / KCH;
+        for (int st = 0; st < nstage; ++st) {
           if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
             fail(33);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem_a + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(smem_b + stage * B_BYTES);
+          const int nk = min(KCH, nkb - st * KCH);
+          const uint32_t a_addr = smem_u32(smem_a + stage * A_STAGE);
+          const uint32_t b_addr = smem_u32(smem_b + stage * B_STAGE);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                           (kb | kk) != 0 ? 1u : 0u);
+          for (int ch = 0; ch < KCH; ++ch) {
+            if (ch < nk) {
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_bf16_pair(d_tmem, sw128_kmajor_desc(a_addr + ch * A_BYTES + kk * 32),
+                               sw128_kmajor_desc(b_addr + ch * B_BYTES + kk * 32), idesc,
+                               (st | ch | kk) != 0 ? 1u : 0u);
+            }
+          }
           umma_commit_pair(&c.empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
