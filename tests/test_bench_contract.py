@@ -1,0 +1,82 @@
+"""The quantities bench.py reports beside its timings, checked on the CPU
+against facts fixed independently of the code that computes them: the FLOP
+count of the layer from its shapes, the kernels one forward launches (as
+listed by the committed ncu launch lists), the bytes a W4A16 expert holds
+(from the weight format: two codes per byte, one bf16 scale per 128
+weights), and the rule that a DRAM traffic figure is reported only while the
+profiled kernel source is unchanged."""
+
+import hashlib
+import json
+import os
+
+import pytest
+
+import bench
+from moe_inputs.configs import CONFIGS
+
+
+def test_gemm_flops_of_the_mid_layer():
+    cfg = CONFIGS["mid"]
+    routed, shared = bench.gemm_flops(cfg)
+    R = 4096 * 6
+    # gate/up: 2 * R * H * 2I; down: 2 * R * I * H
+    assert routed == 2 * R * 2048 * 2 * 1408 + 2 * R * 1408 * 2048 == 425_201_762_304
+    assert shared == 2 * 4096 * 2048 * 2 * 2816 + 2 * 4096 * 2816 * 2048 == 141_733_920_768
+
+
+@pytest.mark.parametrize("name,expected", [
+    # router split + tensor-core logits + top-k, count/rank + scan + scatter,
+    # gate/up + down (shared expert as a second problem), combine
+    ("mid", 9),
+    ("large_prefill", 9),
+    # ... + shared expert by split-K (2 GEMMs + 2 slice sums) + W4A16 (prep +
+    # GEMV) x 2
+    ("decode_w4a16", 15),
+    # ... + token prep + dequantising gate/up and down + bf16 shared gate/up
+    # and down launches
+    ("prefill_w4a16", 12),
+])
+def test_launches_per_step_match_the_launch_lists(name, expected):
+    assert bench.launches_per_step(CONFIGS[name]) == expected
+
+
+def test_launch_list_of_the_mid_layer_has_nine_kernels_per_forward():
+    """The committed launch list names nine distinct kernels of one forward;
+    each appears once per forward (the FFN kernel twice: gate/up and down)."""
+    text = open(os.path.join(bench.ROOT, "profiles", "launches_mid.md")).read()
+    kernels = {"ffn_pair_kernel<GateUp>", "ffn_pair_kernel<Down>", "combine_kernel", "perm_scatter_kernel",
+               "router_topk_kernel", "splitk_gemm_kernel", "perm_scan_kernel", "perm_count_rank_kernel",
+               "router_split_kernel"}
+    for k in kernels:
+        assert f"| {k}" in text, k
+    assert len(kernels) == bench.launches_per_step(CONFIGS["mid"])
+
+
+def test_w4a16_bytes_of_one_touched_expert():
+    import torch
+    cfg = CONFIGS["decode_w4a16"]
+    ids = torch.tensor([[3, 3], [3, 3]])  # one touched expert
+    touched, total = bench.w4a16_bytes(cfg, ids)
+    H, I, Is, T, k = 6144, 2048, 2048, cfg.T, cfg.k
+    codes = (2 * I * H + H * I) // 2            # two 4-bit codes per byte
+    scales = 2 * (2 * I * H + H * I) // 128      # one bf16 per 128 weights
+    shared = 2 * (3 * H * Is)                    # bf16 shared expert
+    acts = 2 * T * H * (2 + 2 * k)
+    assert touched == 1
+    assert codes + scales == 19_464_192
+    assert total == codes + scales + shared + acts
+
+
+def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):
+    src = tmp_path / "kernel.cu"
+    src.write_bytes(b"// kernel v1\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"grouped_ffn_x": {"source": "kernel.cu", "source_sha256_16": sha, "dram_bytes_per_call": 1234}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_from_profile("grouped_ffn_x") == 1234
+    assert bench.traffic_from_profile("grouped_ffn_y") is None
+    src.write_bytes(b"// kernel v2\n")  # the kernel changed after the capture
+    assert bench.traffic_from_profile("grouped_ffn_x") is None
