@@ -110,6 +110,20 @@ def select_topk(logits: torch.Tensor, correction_bias: Optional[torch.Tensor],
     return Selection(ids, weights, s, b, gap)
 
 
+def override_selection(sel: Selection, ids: torch.Tensor, alpha: float,
+                       renorm: bool) -> Selection:
+    """The selection with its ids replaced by ``ids`` (another valid choice,
+    e.g. for a token whose k-th and (k+1)-th biased scores nearly tie).  The
+    emitted weights follow the given ids exactly as for a routed selection
+    ([glm5next] §Numerics): the unbiased scores of those ids, renormalised
+    over them when enabled, then times routed_scaling_factor."""
+    ids = ids.to(torch.int64).cpu()
+    chosen = torch.gather(sel.scores, 1, ids)
+    if renorm:
+        chosen = chosen / chosen.sum(dim=1, keepdim=True)
+    return Selection(ids, alpha * chosen, sel.scores, sel.biased, sel.gap)
+
+
 # --------------------------------------------------------------- permute ----
 
 @dataclass
@@ -227,11 +241,7 @@ def moe_forward(layer, tokens: Optional[Sequence[int]] = None,
     sel = select_topk(router_logits(x, layer.router_w), layer.correction_bias,
                       k, cfg.alpha, cfg.renorm)
     if ids_override is not None:
-        ids = ids_override.to(torch.int64).cpu()
-        chosen = torch.gather(sel.scores, 1, ids)
-        if cfg.renorm:
-            chosen = chosen / chosen.sum(dim=1, keepdim=True)
-        sel = Selection(ids, cfg.alpha * chosen, sel.scores, sel.biased, sel.gap)
+        sel = override_selection(sel, ids_override, cfg.alpha, cfg.renorm)
     perm = permute(sel.ids, E)
 
     R = T * k

@@ -100,6 +100,20 @@ def test_hand_layer_output(hand):
     assert torch.allclose(res.out[0], torch.tensor(hand["layer"]["out"], dtype=f64), atol=1e-14)
 
 
+def test_hand_override_renormalises_the_given_ids(hand):
+    """ids_override: the weights come from the unbiased scores of the given
+    ids, renormalised over those ids before alpha, in the given slot order."""
+    ov = hand["layer_override_renorm"]
+    lay = _hand_layer(hand, alpha=ov["alpha"], renorm=True)
+    res = oracle.moe_forward(lay, ids_override=torch.tensor([ov["ids"]]), keep_hidden=True)
+    assert res.selection.ids[0].tolist() == ov["ids"]
+    assert torch.allclose(res.selection.weights[0], torch.tensor(ov["weights"], dtype=f64), atol=1e-14)
+    # expert 3's routed row holds h3 (rows of expert 0 come first in the permutation)
+    assert res.perm.expert_offsets.tolist() == [0, 1, 1, 1, 2]
+    assert abs(float(res.h_perm[1, 0]) - ov["h3"]) < 1e-16
+    assert torch.allclose(res.out[0], torch.tensor(ov["out"], dtype=f64), atol=1e-14)
+
+
 def test_hand_w4a16_dequant(hand):
     w = hand["w4a16"]
     q = torch.full((1, 64), w["q_fill_byte"], dtype=torch.uint8)

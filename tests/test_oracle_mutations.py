@@ -149,4 +149,27 @@ def test_dropped_shared_expert_is_caught(monkeypatch, hand):
     _expect_fail(pins.test_hand_layer_output, hand)
 
 
+def _override_from_biased(sel, ids, alpha, renorm):      # weights from the biased scores
+    ids = ids.to(torch.int64).cpu()
+    chosen = torch.gather(sel.biased, 1, ids)
+    if renorm:
+        chosen = chosen / chosen.sum(1, keepdim=True)
+    return om.Selection(ids, alpha * chosen, sel.scores, sel.biased, sel.gap)
+
+
+def _override_without_renorm(sel, ids, alpha, renorm):    # renormalisation skipped
+    ids = ids.to(torch.int64).cpu()
+    return om.Selection(ids, alpha * torch.gather(sel.scores, 1, ids), sel.scores, sel.biased, sel.gap)
+
+
+def test_override_weights_from_biased_scores_are_caught(monkeypatch, hand):
+    _patch(monkeypatch, "override_selection", _override_from_biased)
+    _expect_fail(pins.test_hand_override_renormalises_the_given_ids, hand)
+
+
+def test_override_without_renorm_is_caught(monkeypatch, hand):
+    _patch(monkeypatch, "override_selection", _override_without_renorm)
+    _expect_fail(pins.test_hand_override_renormalises_the_given_ids, hand)
+
+
 hand = pins.hand
