@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=CONFIG_NAME,
                     help="layer to time (default: the mid layer the metric is quoted on)")
     ap.add_argument("--graph", action="store_true", help="replay the forward from a captured CUDA graph")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the W4A16 decode-layer measurement added beside the mid layer's line")
     return ap.parse_args(argv)
 
 
@@ -160,23 +162,43 @@ def gemm_flops(cfg):
     return routed, shared
 
 
-def run_cpu_baseline(inp, min_seconds=10.0, max_passes=20):
+def run_cpu_baseline(inp, min_seconds=10.0, max_passes=20, gpu_out=None, gpu_ids=None):
     """The oracle as it stands, on the host cores: whole-layer passes until
-    about `min_seconds` of CPU work (at least one, at most `max_passes`)."""
+    about `min_seconds` of CPU work (at least one, at most `max_passes`).
+    The last pass also checks the timed GPU run's result: expert ids against
+    the oracle's (near-ties, where the k-th and (k+1)-th biased scores are
+    within 1e-6, counted apart) and the layer output within the bf16
+    tolerance max|gpu - oracle| <= 2e-2 max|oracle|."""
     import torch
     import oracle
     cores = torch.get_num_threads()
     t0 = time.perf_counter()
     passes = 0
+    res = None
     while passes < max_passes:
-        oracle.moe_forward(inp)
+        res = oracle.moe_forward(inp)
         passes += 1
         if time.perf_counter() - t0 >= min_seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": passes * inp.cfg.T / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{passes} passes of the full {inp.cfg.name} layer ({inp.cfg.T} tokens each), fp64 torch CPU, "
-                      f"{dt:.1f} s"}
+    line = {"value": passes * inp.cfg.T / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{passes} passes of the full {inp.cfg.name} layer ({inp.cfg.T} tokens each), fp64 torch "
+                      f"CPU, {dt:.1f} s"}
+    if gpu_out is not None and gpu_ids is not None:
+        sel = res.selection
+        tie = sel.gap < 1e-6
+        mism = (gpu_ids.to(torch.int64) != sel.ids).any(dim=1)
+        ok = not bool((mism & ~tie).any())
+        if ok:  # near-tie tokens are re-evaluated with the GPU's (equally valid) selection
+            ref = oracle.moe_forward(inp, ids_override=gpu_ids).out if bool(mism.any()) else res.out
+            err = float((gpu_out.double() - ref).abs().max() / ref.abs().max())
+        else:
+            err = None
+        line["parity"] = {"near_ties": int(tie.sum()), "near_ties_chosen_differently": int((mism & tie).sum()),
+                          "ids_mismatched_outside_near_ties": int((mism & ~tie).sum()),
+                          "out_max_rel_err": err, "tolerance": 2e-2,
+                          "checked": "every token of the timed run's output"}
+    return line
 
 
 def w4a16_bytes(cfg, ids):
@@ -246,6 +268,83 @@ def replica_tokens_per_s(world, tokens_per_rank, ms_per_step):
     """Whole-job throughput of N replicas: every rank processes its own
     tokens each step; the step time is the max over ranks."""
     return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
+# ------------------------------------------------- W4A16 decode layer ----
+
+DECODE_NAME = "decode_w4a16"
+
+
+def measure_decode(dev, iters, clocks, max_over_ranks):
+    """The W4A16 decode layer (T=32, H=6144, E=256, k=8, int4 g128 experts)
+    beside the mid layer's line: its expert FFN call (the HBM-bound part:
+    codes and scales of every touched expert, the bf16 shared expert) and
+    its whole forward, each timed with CUDA events over `iters` calls after
+    warm-up.  The touched experts' codes alone (about 2.9 GB) exceed L2."""
+    import torch
+    import routed_swiglu_experts_b200 as rse
+    cfg, inp = make_inputs(DECODE_NAME)
+    c = cfg
+
+    def mv(t):
+        return None if t is None else t.to(dev)
+    layer = rse.MoELayer(hidden=c.H, num_experts=c.E, top_k=c.k, expert_inter=c.I, shared_inter=c.I_s,
+                         swiglu_limit=c.swiglu_limit, routed_scaling_factor=c.alpha, renormalize=c.renorm,
+                         router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias),
+                         w_gate_up=mv(inp.w_gate_up), w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up),
+                         s_down=mv(inp.s_down), shared_w_gate_up=mv(inp.shared_w_gate_up),
+                         shared_w_down=mv(inp.shared_w_down), max_tokens=c.T)
+    x = inp.x.to(dev)
+    T, k, E, H = c.T, c.k, c.E, c.H
+    R = T * k
+    stream = torch.cuda.current_stream()
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    tw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(R, dtype=torch.int32, device=dev)
+    src = torch.empty(R, dtype=torch.int32, device=dev)
+    w_perm = torch.empty(R, dtype=torch.float32, device=dev)
+    x_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    sh = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    rse.moe_router_topk(layer.cfg, layer.w, x, T, ids, tw, layer.ws)
+    rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
+
+    def ffn():
+        rse.moe_grouped_swiglu_ffn(layer.cfg, layer.w, x_perm, offs, w_perm, T, y_perm, x, sh, layer.ws)
+
+    def fwd():
+        layer.forward(x, out=out)
+
+    res = {}
+    for name, fn in (("ffn", ffn), ("forward", fwd)):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.time()
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark(w0, time.time())
+        res[name] = max_over_ranks(e0.elapsed_time(e1)) / iters
+    assert layer.device_error() == 0
+    touched, nbytes = w4a16_bytes(c, ids.cpu())
+    peaks = measured_peaks()
+    gbs = nbytes / (res["ffn"] / 1e3) / 1e9
+    return {
+        "workload": f"{c.name} MoE layer: T={c.T}, hidden={c.H}, E={c.E}, top_k={c.k}, I={c.I}, I_s={c.I_s}, "
+                    f"int4 group-128 experts (bf16 scales), bf16 shared expert",
+        "forward_ms": res["forward"], "tokens_per_s": c.T / (res["forward"] / 1e3),
+        "ffn_ms": res["ffn"], "ffn_bytes": nbytes, "touched_experts": touched,
+        "ffn_gbs": gbs, "hbm_peak_gbs": peaks["hbm_gbs"], "ffn_frac_of_hbm": gbs / peaks["hbm_gbs"],
+        "peak_source": f"{peaks['source']} HBM copy", "iters": iters,
+        "note": "HBM-bound W4A16 expert FFN call (the decode layer's roofline); "
+                "L2 not flushed: its 2.9 GB of touched codes exceed L2",
+    }
 
 
 # --------------------------------------------------------------- our arm ----
@@ -392,8 +491,11 @@ def bench_ours(args, rank, world, local_rank):
     barrier()
     assert torch.equal(out_host[(args.steps - 1) % 2], out.cpu()), "end-to-end result differs from the device run"
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    clk = clocks.finish()
     assert layer.device_error() == 0
+    decode = None
+    if c.name == CONFIG_NAME and not args.no_decode:
+        decode = measure_decode(dev, max(20, min(args.steps, 200)), clocks, max_over_ranks)
+    clk = clocks.finish()
 
     peaks = measured_peaks()
     routed_f, shared_f = gemm_flops(c)
@@ -434,10 +536,12 @@ def bench_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step(c) * args.steps,
         "clocks": clk,
     })
+    if decode is not None:
+        line["decode_w4a16"] = decode
     if args.graph:
         line["config"]["launch"] = "CUDA graph replay of the forward"
     if rank == 0 and world == 1 and not args.no_cpu_baseline and c.name == CONFIG_NAME:
-        line["cpu_baseline"] = run_cpu_baseline(inp)
+        line["cpu_baseline"] = run_cpu_baseline(inp, gpu_out=out.cpu(), gpu_ids=ids.cpu())
     if graph is not None:
         del graph
     return line

@@ -88,7 +88,8 @@ typedef struct moe_config {
   int32_t shared_inter;          /* I_s (multiple of 8; 0 = no shared expert) */
   float swiglu_limit;            /* L > 0, required (no default); +inf = no
                                     clamp.  gate <- min(gate, L),
-                                    up <- clamp(up, -L, L) */
+                                    up <- clamp(up, -L, L).  W4A16 experts:
+                                    L <= MOE_INT4_MAX_SWIGLU_LIMIT */
   float routed_scaling_factor;   /* alpha: multiplies the routed weights; the
                                     shared expert is added unscaled */
   int32_t renormalize;           /* 1: divide the k unbiased scores by their
@@ -109,7 +110,24 @@ typedef struct moe_weights {
   const void* shared_w_down;     /* bf16 [H, I_s]  (NULL iff I_s == 0) */
 } moe_weights;
 /* W4A16 (int4) packing: byte q[n, c] holds the codes of k = 2c (low nibble)
- * and k = 2c + 1 (high nibble); w[n, k] = (code - 8) * scale[n, k / 128]. */
+ * and k = 2c + 1 (high nibble); w[n, k] = (code - 8) * scale[n, k / 128].
+ *
+ * Range of the W4A16 paths.  Both int4 paths multiply on fp16 tensor-core
+ * operands (fp32 accumulation): the tokens x and the SwiGLU activations h
+ * (already rounded to bf16) are converted to fp16, and the grouped prefill
+ * GEMM also forms the weights (code - 8) * scale in fp16.  Hence:
+ *   - swiglu_limit must be finite and at most MOE_INT4_MAX_SWIGLU_LIMIT, so
+ *     that |h| <= L * L stays finite in fp16 (moe_config_validate returns
+ *     MOE_ERR_UNSUPPORTED otherwise; bf16 experts have no such limit);
+ *   - |x| must stay below 65504 (larger activations become inf; this is not
+ *     checked, the values live on the device);
+ *   - |x| and |h| below about 1e-3, and scales below 2^-14 (prefill GEMM),
+ *     fall into fp16's subnormal range and keep fewer significant bits
+ *     (the GEMV stores half of the activations divided by 16);
+ *   - 8 * |scale| must stay below 65504 (prefill GEMM).
+ * The benchmark layers (x ~ N(0, 1), scales in [0.005, 0.02], L = 7) sit far
+ * inside these bounds. */
+#define MOE_INT4_MAX_SWIGLU_LIMIT 255.0f
 
 /* Human-readable name of a status.  Never NULL. */
 MOE_API const char* moe_status_string(moe_status status);
@@ -220,9 +238,12 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
  * until the process exits), so:
  *   - T * k above MOE_NO_ALLOC_MAX_ROWS returns MOE_ERR_UNSUPPORTED (use
  *     moe_permute with a workspace for larger batches);
- *   - the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing any stream;
+ *   - the first call in each CUDA context (normally the device's primary
+ *     context: once per device) looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it under
+ *     the context's id, so a context created after cudaDeviceReset, or a
+ *     non-primary context made current by the caller, gets its own lookup;
+ *     make that first call before capturing any stream;
  *   - every call shares the array: calls whose kernels may overlap on the
  *     GPU (other streams, other host threads) race and must be ordered on
  *     one stream.  Nothing in it needs clearing between calls.

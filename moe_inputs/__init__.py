@@ -93,7 +93,7 @@ def make_x(cfg: LayerConfig, seed: int = 0, T: Optional[int] = None):
     the token count (the draw is then a different tensor)."""
     T = cfg.T if T is None else T
     g = torch.Generator(device="cpu").manual_seed(seed)
-    x = _normal((T, cfg.H), 1.0, g, "cpu")
+    x = _normal((T, cfg.H), cfg.x_scale, g, "cpu")
     router_w = _normal((cfg.E, cfg.H), 1.0 / math.sqrt(cfg.H), g, "cpu",
                        dtype=torch.float32)
     if cfg.bias_kind == "uniform":

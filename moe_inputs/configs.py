@@ -35,6 +35,7 @@ class LayerConfig:
     zipf_s: float = 1.2
     bias_scale: float = 0.0
     w4a16: bool = False
+    x_scale: float = 1.0        # x ~ N(0, x_scale^2) (1 in every benchmark layer)
 
     @property
     def R(self) -> int:

@@ -27,6 +27,7 @@ MOE_W_BF16 = 0
 MOE_W_INT4_G128 = 1
 MOE_MAX_TOP_K = 16
 MOE_MAX_EXPERTS = 1024
+MOE_INT4_MAX_SWIGLU_LIMIT = 255.0
 
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",

@@ -232,6 +232,9 @@ moe_status moe_config_validate(const moe_config* cfg) {
   if (c.expert_format != MOE_W_BF16 && c.expert_format != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
   if (c.expert_format == MOE_W_INT4_G128 && (c.hidden % 128 != 0 || c.expert_inter % 128 != 0))
     return MOE_ERR_UNSUPPORTED;
+  // the int4 paths feed h to fp16 tensor-core operands: |h| <= L^2 must stay finite in fp16
+  if (c.expert_format == MOE_W_INT4_G128 && !(c.swiglu_limit <= MOE_INT4_MAX_SWIGLU_LIMIT))
+    return MOE_ERR_UNSUPPORTED;
   // TMA strides and boxes: rows of up to 2^31 bytes
   if (static_cast<int64_t>(c.hidden) * 2 >= (int64_t(1) << 31) ||
       static_cast<int64_t>(c.expert_inter) * 2 >= (int64_t(1) << 31))

@@ -12,8 +12,9 @@
 // The array is a file-scope __device__ symbol, so every GPU that loads the
 // library holds it (MOE_NO_ALLOC_SCRATCH_BYTES) until the process exits.
 // Host code may not use the symbol's name as a device address: the first
-// call on each device looks up the real address with cudaGetSymbolAddress
-// (with that device current) and caches it.  Every call reuses the same
+// call in each CUDA context (normally: on each device) looks up the real
+// address with cudaGetSymbolAddress (with that device current) and caches it
+// under the context's id.  Every call reuses the same
 // array, so two calls whose kernels overlap on the GPU (different streams,
 // or different host threads) race on it; order them on one stream.
 #include <mutex>
@@ -35,22 +36,69 @@ static_assert(kNoAllocScratchInts * sizeof(int32_t) == MOE_NO_ALLOC_SCRATCH_BYTE
 // them, so nothing has to be cleared between calls.
 static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocScratchInts];
 
-// Device address of g_perm_scratch per device, looked up once per device.
+// Driver entry points for the context the runtime made current (fetched
+// through the runtime, as for the TMA encoder: no libcuda at link time).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Device address of g_perm_scratch in the current context.  Each CUDA
+// context holds its own copy of the module, so the address is looked up
+// (cudaGetSymbolAddress, with the device current) once per context and
+// cached under the context's process-unique id: a context made after a
+// cudaDeviceReset, or a non-primary context the caller made current, gets an
+// id of its own and its own lookup, never a stale address.
 cudaError_t scratch_address(int32_t** out) {
   static std::mutex mu;
-  static int32_t* addr[64] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static CtxGetCurrentFn get_ctx = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool fns_loaded = false;
+  constexpr int kSlots = 64;
+  static unsigned long long ids[kSlots];
+  static int32_t* addrs[kSlots];
+  static int used = 0;
+  static int next_victim = 0;
+  cudaError_t e = cudaSuccess;
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
+  if (!fns_loaded) {
+    get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    fns_loaded = true;
+  }
+  if (get_ctx == nullptr || get_id == nullptr) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  unsigned long long id = 0;
+  void* p = nullptr;
+  if (ctx == nullptr) {
+    // no context current on this thread yet: the runtime makes the device's
+    // primary context current while it looks the symbol up
     e = cudaGetSymbolAddress(&p, g_perm_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = static_cast<int32_t*>(p);
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
   }
-  *out = addr[dev];
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  for (int i = 0; i < used; ++i)
+    if (ids[i] == id) {
+      *out = addrs[i];
+      return cudaSuccess;
+    }
+  if (p == nullptr) {
+    e = cudaGetSymbolAddress(&p, g_perm_scratch);
+    if (e != cudaSuccess) return e;
+  }
+  int slot = used < kSlots ? used++ : (next_victim++ % kSlots);
+  ids[slot] = id;
+  addrs[slot] = static_cast<int32_t*>(p);
+  *out = addrs[slot];
   return cudaSuccess;
 }
 

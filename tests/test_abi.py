@@ -79,6 +79,11 @@ def mid_cfg(**kw):
     ({"expert_format": _abi.MOE_W_INT4_G128}, _abi.MOE_OK),
     ({"expert_format": _abi.MOE_W_INT4_G128, "expert_inter": 1416}, _abi.MOE_ERR_UNSUPPORTED),
     ({"expert_format": _abi.MOE_W_INT4_G128, "expert_inter": 2048}, _abi.MOE_OK),
+    # int4 experts compute on fp16 operands: |h| <= L^2 must stay finite in fp16
+    ({"expert_format": _abi.MOE_W_INT4_G128, "swiglu_limit": math.inf}, _abi.MOE_ERR_UNSUPPORTED),
+    ({"expert_format": _abi.MOE_W_INT4_G128, "swiglu_limit": 256.0}, _abi.MOE_ERR_UNSUPPORTED),
+    ({"expert_format": _abi.MOE_W_INT4_G128, "swiglu_limit": 255.0}, _abi.MOE_OK),
+    ({"swiglu_limit": 1e30}, _abi.MOE_OK),                # bf16 experts: no such bound
 ])
 def test_config_validation(lib, kw, status):
     if kw.get("expert_format") == _abi.MOE_W_INT4_G128 and "expert_inter" not in kw:

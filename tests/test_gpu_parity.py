@@ -2,9 +2,14 @@
 
 Small layers (spanning several tiles, ragged tails, empty experts, one hot
 expert, exact router ties, the largest supported E and k) are compared in
-full at every stage.  The five benchmark layers are compared at full size:
+full at every stage.  The benchmark layers are compared at full size:
 router ids for every token, the permutation for every slot, and the layer
-output on a seeded sample of tokens.
+output, the shared-expert output and every routed row of the compared
+tokens: all tokens of the mid and decode layers, and on the larger layers a
+sample of at least 1024 tokens chosen per token tile (the first and last
+rows of every tile of every expert, and the rows where a tile's two CTA
+halves meet).  Near-tie counts go into every assertion message and the
+test's printed line.
 
 Bars: expert ids and permutation indices bit-exact (router ids exempt only
 where the oracle's k-th vs (k+1)-th biased-score gap is below 1e-6; those
@@ -53,6 +58,12 @@ EDGE = {
                                  bias_range=0.05, w4a16=True),
     "w4a16_prefill_clamp": LayerConfig("w4a16_prefill_clamp", T=300, H=256, E=4, k=2, I=256, I_s=128,
                                        swiglu_limit=0.5, w4a16=True),
+    # the widest clamp the int4 paths accept (|h| <= L^2 finite in fp16) with
+    # activations 50x the benchmark's: GEMV path, then grouped prefill GEMM
+    "w4a16_wide_limit": LayerConfig("w4a16_wide_limit", T=20, H=256, E=6, k=2, I=128, I_s=128,
+                                    swiglu_limit=255.0, x_scale=50.0, w4a16=True),
+    "w4a16_prefill_wide_limit": LayerConfig("w4a16_prefill_wide_limit", T=300, H=256, E=4, k=2, I=256,
+                                            I_s=128, swiglu_limit=255.0, x_scale=50.0, w4a16=True),
     "shared_small_t32": LayerConfig("shared_small_t32", T=32, H=256, E=4, k=2, I=64, I_s=96, alpha=2.5,
                                     renorm=True),
     "shared_tc_t33": LayerConfig("shared_tc_t33", T=33, H=256, E=4, k=2, I=64, I_s=96),
@@ -203,7 +214,38 @@ def test_tied_router_prefers_lower_id(small_inputs):
 # ------------------------------------------------------ benchmark layers ----
 
 FULL = ["mid", "skewed", "large_prefill", "decode_w4a16", "prefill_w4a16"]
-SAMPLE_TOKENS = {"mid": 96, "skewed": 64, "large_prefill": 12, "decode_w4a16": 12, "prefill_w4a16": 12}
+# layers whose every output row is compared (the oracle runs them in seconds)
+ALL_ROWS = {"mid", "decode_w4a16"}
+TILE_ROWS = 256         # routed rows per token tile of the grouped GEMMs (a CTA pair)
+MIN_SAMPLE = 1024       # tokens compared on the other layers, at least
+
+
+def tile_stratified_tokens(offsets, src, k, T, seed=123):
+    """Tokens whose routed rows sit at the edges of every token tile of every
+    expert: for each expert and each 256-row token tile of it (the last one
+    ragged), the tokens of the tile's first and last row and of the two rows
+    where the tile's halves meet (each CTA of a pair loads one half).  Every
+    expert therefore contributes its first and its last tile, the hot expert
+    of a skewed layer every tile, and, as a token's output row spans every
+    weight-row tile of the down projection, every expert's last weight-row
+    tile is covered too.  Random tokens fill the sample up to MIN_SAMPLE."""
+    off = offsets.tolist()
+    rows = set()
+    for e in range(len(off) - 1):
+        for r0 in range(off[e], off[e + 1], TILE_ROWS):
+            n = min(TILE_ROWS, off[e + 1] - r0)
+            half = (n + 15) // 16 * 8          # token columns of the first CTA (MMA N rounded to 16, halved)
+            for r in (r0, r0 + n - 1, r0 + min(half, n) - 1, r0 + min(half, n - 1)):
+                rows.add(r)
+    src_l = src.tolist()
+    toks = {src_l[r] // k for r in rows}
+    if len(toks) < MIN_SAMPLE:
+        g = torch.Generator().manual_seed(seed)
+        for t in torch.randperm(T, generator=g).tolist():
+            if len(toks) >= MIN_SAMPLE:
+                break
+            toks.add(t)
+    return sorted(toks), sorted(rows)
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -219,31 +261,46 @@ def test_full_size_layer(name):
     sel = oracle.select_topk(oracle.router_logits(inp.x, inp.router_w), inp.correction_bias, cfg.k, cfg.alpha,
                              cfg.renorm)
     n_tie, n_tie_mis = check_ids(st.ids, sel)
+    ties = f"near-ties {n_tie} (gap < 1e-6), of which the GPU chose differently: {n_tie_mis}"
     gpu_ids = st.ids.cpu().to(torch.int64)
     chosen = torch.gather(sel.scores, 1, gpu_ids)
     if cfg.renorm:
         chosen = chosen / chosen.sum(1, keepdim=True)
-    assert torch.allclose(st.topk_w.cpu().double(), cfg.alpha * chosen, rtol=1e-5, atol=1e-7)
+    assert torch.allclose(st.topk_w.cpu().double(), cfg.alpha * chosen, rtol=1e-5, atol=1e-7), ties
 
     # permutation for every slot
     perm = oracle.permute(gpu_ids, cfg.E)
-    assert torch.equal(st.offsets.cpu().long(), perm.expert_offsets)
-    assert torch.equal(st.row_of.cpu().long(), perm.row_of)
-    assert torch.equal(st.src.cpu().long(), perm.src)
+    assert torch.equal(st.offsets.cpu().long(), perm.expert_offsets), ties
+    assert torch.equal(st.row_of.cpu().long(), perm.row_of), ties
+    assert torch.equal(st.src.cpu().long(), perm.src), ties
     src_dev = st.src.long()
     assert torch.equal(st.x_perm, x[src_dev // cfg.k])
     assert torch.equal(st.w_perm, st.topk_w.reshape(-1)[src_dev])
 
-    # layer output on a seeded sample of tokens (with the GPU's ids)
-    g = torch.Generator().manual_seed(123)
-    toks = torch.randperm(cfg.T, generator=g)[:SAMPLE_TOKENS[name]].sort().values
-    res = oracle.moe_forward(inp, tokens=toks.tolist(), ids_override=gpu_ids[toks])
-    err = rel_err(st.out.cpu()[toks], res.out)
-    assert err <= tol_for(cfg), f"{name}: output error {err:.3e}"
+    # layer output: every row, or the tile-stratified token sample (with the GPU's ids)
+    if name in ALL_ROWS:
+        toks = list(range(cfg.T))
+    else:
+        toks, _ = tile_stratified_tokens(perm.expert_offsets, perm.src, cfg.k, cfg.T)
+    tt = torch.tensor(toks, dtype=torch.int64)
+    res = oracle.moe_forward(inp, tokens=toks, ids_override=gpu_ids[tt])
+    tol = tol_for(cfg)
+    what = f"{name}: {len(toks)} of {cfg.T} tokens; {ties}"
+    err = rel_err(st.out.cpu()[tt], res.out)
+    assert err <= tol, f"{what}: output error {err:.3e}"
     if cfg.I_s > 0:
-        assert rel_err(st.shared_out.cpu()[toks], res.shared) <= tol_for(cfg)
+        e_sh = rel_err(st.shared_out.cpu()[tt], res.shared)
+        assert e_sh <= tol, f"{what}: shared-expert error {e_sh:.3e}"
+    # the routed rows of the compared tokens, one by one: y_perm[r] = w_perm[r] * FFN_e(x_t)
+    k = cfg.k
+    slots = (tt[:, None] * k + torch.arange(k)[None, :]).reshape(-1)          # GPU slot ids
+    gpu_rows = st.row_of.cpu().long()[slots]
+    loc_rows = res.perm.row_of                                                # oracle rows, same slot order
+    y_ref = res.y_perm[loc_rows] * st.w_perm.cpu().double()[gpu_rows][:, None]
+    e_y = rel_err(st.y_perm.cpu()[gpu_rows], y_ref)
+    assert e_y <= tol, f"{what}: routed-row error {e_y:.3e}"
     out2 = layer.forward(x)
     torch.cuda.synchronize()
     assert torch.equal(out2, st.out)
     assert layer.device_error() == 0
-    print(f"{name}: near-ties {n_tie} (mismatched {n_tie_mis}), sampled output error {err:.3e}")
+    print(f"{what}; output error {err:.3e}, routed-row error {e_y:.3e}")

@@ -4,8 +4,9 @@ memory and only pass input/output buffers).  Its scratch is a fixed array
 inside the library instead of a caller workspace.
 
 Checked through the C ABI against moe_permute (which takes a workspace) on
-two calls in a row with different shapes, so leftovers of the first call in
-the shared scratch would show up in the second.  Integer and copy outputs
+three calls in a row with different shapes, so leftovers of one call in the
+shared scratch would show up in the next; the last one sits exactly at the
+scratch's limit (T*k == MOE_NO_ALLOC_MAX_ROWS, E == MOE_MAX_EXPERTS).  Integer and copy outputs
 must match bit for bit.  This file is collected last on purpose."""
 
 import pytest
@@ -18,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 def _case(T, H, E, k, seed):
     g = torch.Generator().manual_seed(seed)
-    ids = torch.rand(T, E, generator=g).argsort(dim=1)[:, :k].to(torch.int32)   # k distinct experts
+    ids = torch.rand(T, E, generator=g).topk(k, dim=1).indices.to(torch.int32)   # k distinct experts
     w = torch.rand(T, k, generator=g)
     x = torch.randn(T, H, generator=g).to(torch.bfloat16)
     cfg = _abi.make_config(H, E, k, 64, 0, 7.0, 1.0, False)
@@ -36,7 +37,12 @@ def _outputs(T, H, E, k):
 def test_no_alloc_permute_matches_workspace_permute():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
-    for (T, H, E, k, seed) in [(4096, 2048, 64, 6, 0), (333, 200, 5, 3, 1)]:
+    # the mid layer's shape, a ragged small one, then the scratch's limit:
+    # T * k == MOE_NO_ALLOC_MAX_ROWS with E == MOE_MAX_EXPERTS uses every
+    # (chunk, expert) count slot and the last per-slot rank
+    limit_T = _abi.MOE_NO_ALLOC_MAX_ROWS // 8
+    for (T, H, E, k, seed) in [(4096, 2048, 64, 6, 0), (333, 200, 5, 3, 1),
+                               (limit_T, 64, _abi.MOE_MAX_EXPERTS, 8, 2)]:
         cfg, ids, w, x = _case(T, H, E, k, seed)
         ws = torch.empty(_abi.moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
         _abi.moe_workspace_init(ws)
