@@ -214,9 +214,9 @@ def w4a16_bytes(cfg, ids):
 
 def launches_per_step(cfg):
     """Kernels one forward launches: router 3 (weight split, tensor-core
-    logits, top-k), permute 3 (count/rank, scan, scatter), combine 1, plus the
-    expert FFN path."""
-    n = 7
+    logits, top-k), permute 2 (count/rank with the scan in its last block,
+    scatter), combine 1, plus the expert FFN path."""
+    n = 6
     small_shared = cfg.I_s > 0 and cfg.T <= 32  # split-K GEMMs + slice sums for the shared expert
     shared = (4 if small_shared else 2) if cfg.I_s > 0 else 0
     if cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E:

@@ -246,10 +246,12 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
  *     make that first call before capturing any stream;
  *   - every call shares the array: calls whose kernels may overlap on the
  *     GPU (other streams, other host threads) race and must be ordered on
- *     one stream.  Nothing in it needs clearing between calls.
+ *     one stream.  Nothing in it needs clearing between calls: the one
+ *     word that must start at zero (the count kernel's ticket counter) is
+ *     zero when the library loads and every call leaves it at zero.
  * Never calls cudaMalloc / cudaFree or any allocating routine. */
 #define MOE_NO_ALLOC_MAX_ROWS 131072
-#define MOE_NO_ALLOC_SCRATCH_BYTES 786432
+#define MOE_NO_ALLOC_SCRATCH_BYTES 786688
 MOE_API moe_status moe_permute_no_alloc(const moe_config* cfg, const int32_t* topk_ids,
                                         const float* topk_w, const void* x, int32_t T,
                                         int32_t* expert_offsets, int32_t* row_of, int32_t* src,

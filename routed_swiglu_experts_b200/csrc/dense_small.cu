@@ -55,12 +55,12 @@ __global__ void __launch_bounds__(256)
 
 // K slices so that (column tiles x slices) fills the SMs in one wave, each
 // slice at least 4 k-blocks of 64.
-int splits_for(int N, int K, int num_sms) {
+int splits_for(int N, int K, int T, int num_sms) {
   const int n_tiles = (N + kMmaN - 1) / kMmaN;
   int s = std::max(1, num_sms / n_tiles);
   s = std::min(s, kDenseSmallMaxSplits);
   s = std::min(s, std::max(1, (K / 64) / 4));
-  return splitk_actual_splits(K, 1, s);
+  return splitk_actual_splits(K, 1, kMmaN, T, s);
 }
 
 }  // namespace
@@ -76,7 +76,7 @@ size_t dense_small_part_floats(int H, int Is) {
 cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const void* w_gu, const void* w_d, float L,
                                    float* part, void* h_s, void* out, int32_t* err, int num_sms, cudaStream_t stream) {
   // gate/up: [T, H] x [2 I_s, H]^T
-  int S = splits_for(2 * Is, H, num_sms);
+  int S = splits_for(2 * Is, H, T, num_sms);
   cudaError_t e = launch_splitk_gemm(x, T, H, w_gu, 1, 2 * Is, kMmaN, S, part, err, num_sms, stream);
   if (e != cudaSuccess) return e;
   dense_small_finish_kernel<<<(T * Is / 4 + 255) / 256, 256, 0, stream>>>(part, S, T, 2 * Is, 1, Is, L,
@@ -84,7 +84,7 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // down: [T, I_s] x [H, I_s]^T
-  S = splits_for(H, Is, num_sms);
+  S = splits_for(H, Is, T, num_sms);
   e = launch_splitk_gemm(h_s, T, Is, w_d, 1, H, kMmaN, S, part, err, num_sms, stream);
   if (e != cudaSuccess) return e;
   dense_small_finish_kernel<<<(T * H / 4 + 255) / 256, 256, 0, stream>>>(part, S, T, H, 0, H, 0.f,

@@ -53,6 +53,7 @@ T* at(void* ws, size_t off) {
 
 int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 int32_t* tile_queue(void* ws, TileQueueSlot slot) { return reinterpret_cast<WsHeader*>(ws)->tile_queue + slot; }
+int32_t* perm_ticket(void* ws) { return &reinterpret_cast<WsHeader*>(ws)->perm_done; }
 
 bool is_int4(const moe_config& cfg) { return cfg.expert_format == MOE_W_INT4_G128; }
 
@@ -282,7 +283,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const flo
   if (T == 0) return MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
   return from_cuda(launch_permute(*cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm,
-                                  at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), stream));
+                                  at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), perm_ticket(ws),
+                                  stream));
 }
 
 moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weights* w, const void* x_perm,
@@ -340,7 +342,8 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   float* w_perm = at<float>(ws, L.w_perm);
   void* x_perm = at<void>(ws, L.x_perm);
   MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, at<int32_t>(ws, L.src), w_perm, x_perm,
-                              at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), stream));
+                              at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), perm_ticket(ws),
+                              stream));
   void* y_perm = at<void>(ws, L.y_perm);
   const bool shared = cfg->shared_inter > 0;
   void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;

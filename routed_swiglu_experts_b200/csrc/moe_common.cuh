@@ -20,7 +20,10 @@ struct WsHeader {
   // per kernel: zero when a launch starts, reset to zero by the last CTA
   // pair of every launch.
   int32_t tile_queue[8];
-  int32_t pad[54];
+  // Ticket counter of the permute's count blocks: zero when a launch starts,
+  // reset to zero by the block that takes the last ticket.
+  int32_t perm_done;
+  int32_t pad[53];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 enum TileQueueSlot { kQueueGateUp = 0, kQueueDown = 2, kQueueInt4GateUp = 4, kQueueInt4Down = 6 };

@@ -31,16 +31,19 @@ inline int router_mma_n(int E) { return std::min(256, (E + 15) / 16 * 16); }
 struct RouterPlan {
   int ks;  // k-splits of the logits GEMM (partials summed by the top-k kernel)
 };
-RouterPlan router_plan(int T, int E, int H);
+RouterPlan router_plan(int T, int E, int H, int num_sms);
 size_t router_partial_floats(int Tmax, int E);
 size_t router_topk_smem(int E);
 // Split-K tensor-core GEMM with fp32 partials part[s][rows][N] over `parts`
 // passes of K (B slice p per pass); n_mma: MMA N, a multiple of 16 <= 256.
 cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, int parts, int N, int n_mma,
                                int k_splits, float* part, int32_t* err, int num_sms, cudaStream_t stream);
-int splitk_actual_splits(int K, int parts, int k_splits);
+// K steps of one tile's full reduction (all B slices of a step share a stage
+// when n_mma is small) and the split count a request of k_splits becomes.
+int splitk_steps(int K, int parts, int n_mma, int rows);
+int splitk_actual_splits(int K, int parts, int n_mma, int rows, int k_splits);
 cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStream_t stream);
-int router_actual_splits(int H, int k_splits);
+int router_actual_splits(int T, int E, int H, int k_splits);
 cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
                                int32_t* err, int num_sms, cudaStream_t stream);
 cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const void* x, int T, int32_t* ids,
@@ -49,9 +52,11 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
 // Permute: slots per counting block.
 constexpr int kPermChunk = 2048;
 inline int perm_blocks(int R) { return std::max(1, (R + kPermChunk - 1) / kPermChunk); }
+// block_base: [perm_blocks(T*k) * E] scratch; local_rank: [T*k] scratch;
+// done: a ticket counter that is zero before the launch and left at zero.
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
                            int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
-                           int32_t* block_base, int32_t* local_rank, cudaStream_t stream);
+                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream);
 
 cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
                            const void* shared_out, int T, void* out, cudaStream_t stream);

@@ -1,12 +1,15 @@
 // Token sort / permute by expert ("Module glm5next_mlp", MOE_MODULE: the
 // token sort / permute / unpermute kernels) as a deterministic stable
-// counting sort of the slots i = t*k + j:
+// counting sort of the slots i = t*k + j, in two launches:
 //   1. per 2048-slot chunk: per-expert counts, and each slot's rank among the
 //      earlier slots of its chunk with the same expert (warp match + popc);
-//   2. one block: per-(chunk, expert) bases = expert offset + earlier chunks;
-//   3. scatter: row = base + rank; row_of / src / w_perm, and the 16-byte
+//      the last chunk block to finish (a ticket counter it resets to zero)
+//      turns the counts into per-(chunk, expert) bases = expert offset +
+//      earlier chunks, and writes the expert offsets;
+//   2. scatter: row = base + rank; row_of / src / w_perm, and the 16-byte
 //      vector gather of the token's hidden row into x_perm.
-// No atomics decide an order, so the result is identical run to run.
+// No atomic decides an order (the ticket only picks which block scans), so
+// the result is identical run to run.
 #include "moe_internal.h"
 
 namespace moe {
@@ -17,11 +20,39 @@ constexpr int kPermWarps = 8;
 constexpr int kPermIters = kPermChunk / (kPermWarps * 32);  // 8 slots per lane
 static_assert(kPermIters * kPermWarps * 32 == kPermChunk, "chunk split");
 
-// dynamic smem: cnt[kPermWarps][E]
+// Count tables of at most this many (chunk, expert) entries are scanned in
+// shared memory by the last block; larger ones column by column in global.
+constexpr int kScanSmemEntries = 16384;
+
+// Exclusive prefix over the chunks of every expert column of cnt[nb][E]
+// (chunk-major), in place; tot[e] = the column total.  Run by one block.
+__device__ void scan_columns_global(int32_t* __restrict__ cnt, int nb, int E, int32_t* tot) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int b0 = 0; b0 < nb; b0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = b0 + j < nb ? __ldcg(cnt + static_cast<size_t>(b0 + j) * E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (b0 + j < nb) {
+          cnt[static_cast<size_t>(b0 + j) * E + e] = run;
+          run += v[j];
+        }
+    }
+    tot[e] = run;
+  }
+}
+
+// dynamic smem: max(cnt[kPermWarps][E], table[nb][E] when nb * E <= kScanSmemEntries)
 __global__ void __launch_bounds__(kPermWarps * 32)
     perm_count_rank_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* __restrict__ block_base,
-                           int32_t* __restrict__ local_rank) {
+                           int32_t* __restrict__ local_rank, int32_t* __restrict__ offsets,
+                           int32_t* __restrict__ done) {
   extern __shared__ int32_t cnt[];
+  __shared__ int32_t tot[MOE_MAX_EXPERTS];
+  __shared__ int32_t wsum[kPermWarps];
+  __shared__ int s_last;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int j = threadIdx.x; j < kPermWarps * E; j += blockDim.x) cnt[j] = 0;
   __syncthreads();
@@ -61,56 +92,71 @@ __global__ void __launch_bounds__(kPermWarps * 32)
     const int i = base + it * 32 + lane;
     if (i < R) local_rank[i] = wcnt[idv[it]] + rank[it];
   }
-}
 
-// One block of 1024 threads.  block_base[b][e] (chunk counts) becomes the
-// first routed row of chunk b's slots of expert e; offsets[0..E] written.
-__global__ void __launch_bounds__(1024)
-    perm_scan_kernel(int32_t* __restrict__ block_base, int nblocks, int E, int32_t* __restrict__ offsets) {
-  __shared__ int32_t tot[MOE_MAX_EXPERTS];
-  __shared__ int32_t wsum[32];
-  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblocks; ++b) {
-      const int c = block_base[static_cast<size_t>(b) * E + e];
-      block_base[static_cast<size_t>(b) * E + e] = run;
-      run += c;
+  // the last block to get here turns every chunk's counts into bases
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(done, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int nb = gridDim.x;
+  const int n = nb * E;
+  if (n <= kScanSmemEntries) {
+    int32_t* tab = cnt;  // the chunk's counts are no longer needed
+    for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = __ldcg(block_base + i);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int run = 0;
+      for (int b = 0; b < nb; ++b) {
+        const int c = tab[b * E + e];
+        tab[b * E + e] = run;
+        run += c;
+      }
+      tot[e] = run;
     }
-    tot[e] = run;
+  } else {
+    scan_columns_global(block_base, nb, E, tot);
   }
   __syncthreads();
-  // exclusive scan of tot[0..E) (E <= 1024: one element per thread)
-  const int v = tid < E ? tot[tid] : 0;
-  int incl = v;
+  // exclusive scan of the expert totals (E <= 1024: 4 consecutive per thread)
+  constexpr int kPer = MOE_MAX_EXPERTS / (kPermWarps * 32);
+  int v[kPer];
+  int local = 0;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
+  for (int j = 0; j < kPer; ++j) {
+    const int e = threadIdx.x * kPer + j;
+    v[j] = e < E ? tot[e] : 0;
+    local += v[j];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    int s = wsum[lane];
+  int before = incl - local;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+  __syncthreads();  // every thread has read tot[] for its own entries
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += o;
+  for (int j = 0; j < kPer; ++j) {
+    const int e = threadIdx.x * kPer + j;
+    if (e < E) {
+      offsets[e] = before;
+      tot[e] = before;
     }
-    wsum[lane] = s;  // inclusive over warps
+    before += v[j];
   }
+  if (threadIdx.x == kPermWarps * 32 - 1) offsets[E] = before;  // = R
   __syncthreads();
-  const int excl = incl - v + (warp > 0 ? wsum[warp - 1] : 0);
-  if (tid < E) {
-    offsets[tid] = excl;
-    tot[tid] = excl;
+  if (n <= kScanSmemEntries) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) block_base[i] = cnt[i] + tot[i % E];
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) block_base[i] += tot[i % E];
   }
-  if (tid == E - 1) offsets[E] = excl + v;
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int o = tot[e];
-    for (int b = 0; b < nblocks; ++b) block_base[static_cast<size_t>(b) * E + e] += o;
-  }
+  if (threadIdx.x == 0) *done = 0;  // ready for the next launch
 }
 
 // One warp per slot: routed row, inverse maps, weight, and the hidden row.
@@ -148,16 +194,17 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
                            int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
-                           int32_t* block_base, int32_t* local_rank, cudaStream_t stream) {
+                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream) {
   const int E = cfg.num_experts, k = cfg.top_k, H = cfg.hidden;
   const int R = T * k;
   const int nb = perm_blocks(R);
-  const size_t smem = static_cast<size_t>(kPermWarps) * E * sizeof(int32_t);
+  const size_t n = static_cast<size_t>(nb) * E;
+  const size_t smem = std::max(static_cast<size_t>(kPermWarps) * E, n <= kScanSmemEntries ? n : 0) * sizeof(int32_t);
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(perm_count_rank_kernel),
-                                   kPermWarps * MOE_MAX_EXPERTS * static_cast<int>(sizeof(int32_t)));
+                                   static_cast<int>(std::max(kPermWarps * MOE_MAX_EXPERTS, kScanSmemEntries) *
+                                                    sizeof(int32_t)));
   if (e != cudaSuccess) return e;
-  perm_count_rank_kernel<<<nb, kPermWarps * 32, smem, stream>>>(ids, R, E, block_base, local_rank);
-  perm_scan_kernel<<<1, 1024, 0, stream>>>(block_base, nb, E, offsets);
+  perm_count_rank_kernel<<<nb, kPermWarps * 32, smem, stream>>>(ids, R, E, block_base, local_rank, offsets, done);
   perm_scatter_kernel<<<(R + 7) / 8, 256, 0, stream>>>(ids, topk_w, static_cast<const __nv_bfloat16*>(x), R, k, E,
                                                        H, block_base, local_rank, row_of, src, w_perm,
                                                        static_cast<__nv_bfloat16*>(x_perm));

@@ -26,14 +26,17 @@ namespace moe {
 namespace {
 
 constexpr int kNoAllocMaxChunks = MOE_NO_ALLOC_MAX_ROWS / kPermChunk;
+constexpr size_t kNoAllocTicketInts = 64;  // one ticket word, padded to 256 bytes
 constexpr size_t kNoAllocBlockBaseInts = static_cast<size_t>(kNoAllocMaxChunks) * MOE_MAX_EXPERTS;
-constexpr size_t kNoAllocScratchInts = kNoAllocBlockBaseInts + MOE_NO_ALLOC_MAX_ROWS;
+constexpr size_t kNoAllocScratchInts = kNoAllocTicketInts + kNoAllocBlockBaseInts + MOE_NO_ALLOC_MAX_ROWS;
 static_assert(MOE_NO_ALLOC_MAX_ROWS % kPermChunk == 0, "whole chunks");
 static_assert(kNoAllocScratchInts * sizeof(int32_t) == MOE_NO_ALLOC_SCRATCH_BYTES, "documented size");
 
-// [kNoAllocMaxChunks * E] chunk counts / bases, then [T*k] in-chunk ranks.
-// Both parts are fully written by the count kernel before anything reads
-// them, so nothing has to be cleared between calls.
+// [64] the count blocks' ticket counter (word 0), then [kNoAllocMaxChunks * E]
+// chunk counts / bases, then [T*k] in-chunk ranks.  The counter is zero when
+// the module loads and every call leaves it at zero; the other two parts are
+// fully written by the count kernel before anything reads them.  So nothing
+// has to be cleared between calls.
 static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocScratchInts];
 
 // Driver entry points for the context the runtime made current (fetched
@@ -123,9 +126,10 @@ extern "C" MOE_API moe_status moe_permute_no_alloc(const moe_config* cfg, const 
   if (T == 0) return MOE_OK;
   int32_t* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
-  int32_t* block_base = scratch;
-  int32_t* local_rank = scratch + kNoAllocBlockBaseInts;
+  int32_t* ticket = scratch;
+  int32_t* block_base = scratch + kNoAllocTicketInts;
+  int32_t* local_rank = block_base + kNoAllocBlockBaseInts;
   const cudaError_t e = launch_permute(*cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm,
-                                       block_base, local_rank, stream);
+                                       block_base, local_rank, ticket, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -1,7 +1,7 @@
 // Router: the fp32 logits GEMM runs on the tensor cores (splitk_gemm.cu, three
 // passes over K) on an exact bf16 split of the fp32 weight; here are the split
-// and the warp-per-token sigmoid + biased top-k with an fp64 re-rank of
-// near-ties.
+// and the sigmoid + biased top-k (per token: one thread when the order is
+// certain, one warp with an fp64 re-rank of near-ties when it is not).
 //
 // "Module glm5next_mlp" §Numerics: sigmoid score; the correction bias steers
 // selection only; the emitted weight is the unbiased score times
@@ -128,79 +128,46 @@ __device__ __forceinline__ double exact_biased_one(const __nv_bfloat16* __restri
   return 1.0 / (1.0 + exp(-a0)) + (bias != nullptr ? static_cast<double>(bias[e0]) : 0.0);
 }
 
-// One warp per token (with one token per block, every warp of the block
-// shares that token's fp64 scores).
-//  1. s = sigmoid(sum of the partial logits), b = s + bias (fp32).
-//  2. Extract experts in (b desc, id asc) order: the top k+1, and, while the
-//     k-th/(k+1)-th boundary is a near-tie, every further expert that
-//     continues the run of adjacent gaps below tau.
-//  3. Any run ("cluster") of adjacent gaps below tau that reaches into the
-//     top k is re-ordered by fp64 biased scores (ties to the lower id); order
-//     between clusters is certain because tau is far above the fp32 error.
-//  4. Emit ids and alpha * s (renormalised over the k if asked).
-__global__ void __launch_bounds__(kTopkWarps * 32)
-    router_topk_kernel(const float* __restrict__ part, int KS, const __nv_bfloat16* __restrict__ x,
-                       const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H,
-                       int k, float alpha, int renorm, float tau, int tpb, int32_t* __restrict__ ids_out,
-                       float* __restrict__ w_out) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t0 = blockIdx.x * tpb;
-  const size_t pw = topk_smem_per_warp(E);
+// A warp's scratch for selecting one token's experts (see
+// topk_smem_per_warp): fp32 unbiased and biased scores of every expert, the
+// experts extracted in order with their biased scores, fp64 scores of
+// near-tie clusters, and the k chosen ids.
+struct WarpArea {
+  double* v64;
+  float* s;
+  float* b;
+  float* lv;
+  int* lst;
+  int* res;
+};
 
-  // 1. all threads of the block: sum the split-H partial logits of the
-  //    block's tpb tokens, s = sigmoid, b = s + bias, into the token's warp area
-  for (int idx = threadIdx.x; idx < tpb * E; idx += blockDim.x) {
-    const int w = idx / E, e = idx - w * E;
-    const int tt = t0 + w;
-    if (tt < T) {
-      // slices are added in ascending order, loaded 8 at a time
-      float l = 0.f;
-      const float* pp = part + static_cast<size_t>(tt) * E + e;
-      const size_t slice = static_cast<size_t>(T) * E;
-      int ks = 0;
-      for (; ks + 8 <= KS; ks += 8) {
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __ldg(pp + (ks + j) * slice);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) l += v[j];
-      }
-      for (; ks < KS; ++ks) l += __ldg(pp + ks * slice);
-      const float sv = 1.f / (1.f + expf(-l));
-      float* sw = reinterpret_cast<float*>(smem_raw + pw * w + static_cast<size_t>(E) * 8);
-      sw[e] = sv;
-      sw[E + e] = sv + (bias != nullptr ? bias[e] : 0.f);
-    }
-  }
-  __syncthreads();
-  const bool coop = tpb == 1;  // block-uniform
-  const int t = t0 + (coop ? 0 : warp);
-  if (coop ? t >= T : (warp >= tpb || t >= T)) return;
-  const bool owner = !coop || warp == 0;
+__device__ __forceinline__ WarpArea warp_area(unsigned char* base, int E) {
+  WarpArea w;
+  w.v64 = reinterpret_cast<double*>(base);
+  w.s = reinterpret_cast<float*>(base + static_cast<size_t>(E) * 8);
+  w.b = w.s + E;
+  w.lv = w.b + E;
+  w.lst = reinterpret_cast<int*>(w.lv + E);
+  w.res = w.lst + E;
+  return w;
+}
 
-  unsigned char* base = smem_raw + pw * (coop ? 0 : warp);
-  double* v64 = reinterpret_cast<double*>(base);
-  float* s_sm = reinterpret_cast<float*>(base + static_cast<size_t>(E) * 8);
-  float* b_sm = s_sm + E;
-  float* lv = b_sm + E;
-  int* lst = reinterpret_cast<int*>(lv + E);
-  int* res = lst + E;
+// Phase 2 (one warp, w.s and w.b filled): extract experts in (b desc, id
+// asc) order -- the top k+1, and, while the k-th/(k+1)-th boundary is a
+// near-tie, every further expert that continues the run of adjacent gaps
+// below tau.  Returns how many were extracted; res[0..k) = the first k.
+__device__ int warp_extract(const WarpArea& w, int E, int k, float tau, int lane) {
   const int nm = (E + 31) / 32;  // entries per lane: e = lane + 32 m
-
-  // 2. ordered extraction (the owner warp)
-  __shared__ int s_n;
-  int n = 0;
-  if (owner) {
   uint32_t taken = 0;
   const int k1 = min(k + 1, E);
+  int n = 0;
   while (n < E) {
     float v = -INFINITY;
     int id = 0x7fffffff;
     for (int m = 0; m < nm; ++m) {
       const int e = lane + 32 * m;
       if (e < E && !((taken >> m) & 1u)) {
-        const float bv = b_sm[e];
+        const float bv = w.b[e];
         if (bv > v || (bv == v && e < id)) {
           v = bv;
           id = e;
@@ -209,60 +176,43 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     }
     warp_argmax(v, id);
     if (n >= k1) {  // past k+1: only while the boundary run continues
-      const bool boundary_tie = lv[k - 1] - lv[k] < tau;
-      if (!boundary_tie || !(lv[n - 1] - v < tau)) break;
+      const bool boundary_tie = w.lv[k - 1] - w.lv[k] < tau;
+      if (!boundary_tie || !(w.lv[n - 1] - v < tau)) break;
     }
     if ((id & 31) == lane) taken |= 1u << (id / 32);
     if (lane == 0) {
-      lst[n] = id;
-      lv[n] = v;
+      w.lst[n] = id;
+      w.lv[n] = v;
     }
     __syncwarp();
     ++n;
   }
-  if (lane < k) res[lane] = lst[lane];
-  if (coop && lane == 0) s_n = n;
+  if (lane < k) w.res[lane] = w.lst[lane];
   __syncwarp();
-  }
+  return n;
+}
 
-  // 3. fp64 re-order of the near-tie clusters that reach into the top k.
-  //    Cluster [a, b]: a maximal run of adjacent gaps below tau starting at
-  //    a < k.  With one token per block all warps first compute the fp64
-  //    scores of every clustered entry, then the owner orders them.
-  const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
-  if (coop) {
-    __syncthreads();
-    n = s_n;
-    for (int i = warp; i < n; i += kTopkWarps) {
-      // entry i needs an fp64 score if its cluster has two entries or more
-      int a = 0, b = 0;
-      while (true) {
-        b = a;
-        while (b + 1 < n && lv[b] - lv[b + 1] < tau) ++b;
-        if (i <= b || b + 1 >= k) break;
-        a = b + 1;
-      }
-      if (a < k && i >= a && i <= b && b > a) {
-        const double d = exact_biased_one(xr, wr, bias, H, lane, lst[i]);
-        if (lane == 0) v64[i] = d;
-      }
-    }
-    __syncthreads();
-    if (!owner) return;
-  }
+// Phase 3 (one warp): re-order by fp64 biased scores every near-tie cluster
+// -- a maximal run [a, b] of adjacent gaps below tau with a < k -- ties to
+// the lower id.  With have_v64 the fp64 scores of the clustered entries are
+// already in w.v64; otherwise this warp computes them.  Order between
+// clusters is certain: tau is far above the fp32 error of the logits.
+__device__ void warp_rerank(const WarpArea& w, int n, const __nv_bfloat16* __restrict__ xr,
+                            const float* __restrict__ wr, const float* __restrict__ bias, int H, int k, float tau,
+                            bool have_v64, int lane) {
   int a = 0;
   while (a < k) {
     int b = a;
-    while (b + 1 < n && lv[b] - lv[b + 1] < tau) ++b;
+    while (b + 1 < n && w.lv[b] - w.lv[b + 1] < tau) ++b;
     if (b > a) {
-      if (!coop) {
+      if (!have_v64) {
         for (int i = a; i <= b; i += 2) {
           const int j = min(i + 1, b);
           double d0, d1;
-          exact_biased_pair(xr, wr, bias, H, lane, lst[i], lst[j], d0, d1);
+          exact_biased_pair(xr, wr, bias, H, lane, w.lst[i], w.lst[j], d0, d1);
           if (lane == 0) {
-            v64[i] = d0;
-            v64[j] = d1;
+            w.v64[i] = d0;
+            w.v64[j] = d1;
           }
         }
       }
@@ -274,8 +224,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         int id = 0x7fffffff;
         for (int i = a + lane, m = 0; i <= b; i += 32, ++m) {
           if (!((ctaken >> m) & 1u)) {
-            const double bv = v64[i];
-            const int e = lst[i];
+            const double bv = w.v64[i];
+            const int e = w.lst[i];
             if (bv > v || (bv == v && e < id)) {
               v = bv;
               id = e;
@@ -284,37 +234,272 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         }
         warp_argmax(v, id);
         for (int i = a + lane, m = 0; i <= b; i += 32, ++m)
-          if (lst[i] == id) ctaken |= 1u << m;
-        if (lane == 0) res[a + sidx] = id;
+          if (w.lst[i] == id) ctaken |= 1u << m;
+        if (lane == 0) w.res[a + sidx] = id;
       }
       __syncwarp();
     }
     a = b + 1;
   }
+}
 
-  // 4. emitted weights from the unbiased fp32 scores
+// Phase 4 (one warp): ids and alpha * s of the chosen experts from the
+// unbiased fp32 scores, renormalised over the k (in selection order) if asked.
+__device__ void warp_emit(const WarpArea& w, int k, float alpha, int renorm, int lane, int32_t* __restrict__ ids_row,
+                          float* __restrict__ w_row) {
   float wsum = 0.f;
-  for (int r = 0; r < k; ++r) wsum += s_sm[res[r]];
+  for (int r = 0; r < k; ++r) wsum += w.s[w.res[r]];
   if (lane < k) {
-    const int id = res[lane];
-    const float sv = s_sm[id];
-    ids_out[static_cast<size_t>(t) * k + lane] = id;
-    w_out[static_cast<size_t>(t) * k + lane] = renorm ? (sv / wsum) * alpha : sv * alpha;
+    const int id = w.res[lane];
+    const float sv = w.s[id];
+    ids_row[lane] = id;
+    w_row[lane] = renorm ? (sv / wsum) * alpha : sv * alpha;
   }
+}
+
+// Few tokens: one token per block of kTopkWarps warps.  All threads sum the
+// token's K-slice partial logits (slices in ascending order) into s and b;
+// warp 0 extracts; every warp computes fp64 scores of the clustered entries;
+// warp 0 re-orders and emits.
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    router_topk_coop_kernel(const float* __restrict__ part, int KS, const __nv_bfloat16* __restrict__ x,
+                            const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H, int k,
+                            float alpha, int renorm, float tau, int32_t* __restrict__ ids_out,
+                            float* __restrict__ w_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ int s_n;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x;
+  const WarpArea w = warp_area(smem_raw, E);
+  const size_t slice = static_cast<size_t>(T) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float l = 0.f;
+    const float* pp = part + static_cast<size_t>(t) * E + e;
+    int ks = 0;
+    for (; ks + 8 <= KS; ks += 8) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __ldg(pp + (ks + j) * slice);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) l += v[j];
+    }
+    for (; ks < KS; ++ks) l += __ldg(pp + ks * slice);
+    const float sv = 1.f / (1.f + expf(-l));
+    w.s[e] = sv;
+    w.b[e] = sv + (bias != nullptr ? bias[e] : 0.f);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int n = warp_extract(w, E, k, tau, lane);
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const __nv_bfloat16* xr = x + static_cast<size_t>(t) * H;
+  for (int i = warp; i < n; i += kTopkWarps) {
+    // entry i needs an fp64 score if its cluster has two entries or more
+    int a = 0, b = 0;
+    while (true) {
+      b = a;
+      while (b + 1 < n && w.lv[b] - w.lv[b + 1] < tau) ++b;
+      if (i <= b || b + 1 >= k) break;
+      a = b + 1;
+    }
+    if (a < k && i >= a && i <= b && b > a) {
+      const double d = exact_biased_one(xr, wr, bias, H, lane, w.lst[i]);
+      if (lane == 0) w.v64[i] = d;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  warp_rerank(w, n, xr, wr, bias, H, k, tau, true, lane);
+  warp_emit(w, k, alpha, renorm, lane, ids_out + static_cast<size_t>(t) * k, w_out + static_cast<size_t>(t) * k);
+}
+
+// Many tokens: a block takes `tb` consecutive tokens (one per thread of its
+// first tb threads).
+//  1. All 256 threads sum the block's K-slice partial logits -- contiguous
+//     rows, 16-byte loads, slices in ascending order -- into shared memory.
+//  2. Each token's thread walks its E experts in id order, s = sigmoid(l),
+//     b = s + bias, keeping the NS largest b (desc, ties to the lower id: an
+//     expert enters only by beating the smallest kept value) in registers.
+//  3. If no two adjacent values among the top k+1 are closer than tau, the
+//     order is certain and the thread emits the k ids and weights.  Otherwise
+//     the token's warp takes it: s and b into the warp's scratch, then the
+//     same extraction, fp64 re-order of near-tie clusters and emission as
+//     the few-token kernel.
+constexpr int kRowsThreads = 256;
+
+template <int NS>
+__device__ __forceinline__ void keep_top(float (&val)[NS], float (&sv)[NS], int (&id)[NS], float b, float s, int e) {
+  // val is sorted descending; b > val[NS-1]: insert it after every kept value
+  // >= b (those have lower ids), shifting the smaller ones down
+#pragma unroll
+  for (int j = NS - 1; j > 0; --j) {
+    if (val[j - 1] < b) {
+      val[j] = val[j - 1];
+      sv[j] = sv[j - 1];
+      id[j] = id[j - 1];
+    } else if (val[j] < b) {
+      val[j] = b;
+      sv[j] = s;
+      id[j] = e;
+    }
+  }
+  if (val[0] < b) {
+    val[0] = b;
+    sv[0] = s;
+    id[0] = e;
+  }
+}
+
+template <int NS>
+__global__ void __launch_bounds__(kRowsThreads)
+    router_topk_rows_kernel(const float* __restrict__ part, int KS, const __nv_bfloat16* __restrict__ x,
+                            const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H, int k,
+                            float alpha, int renorm, float tau, int tb, int32_t* __restrict__ ids_out,
+                            float* __restrict__ w_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const size_t pw = topk_smem_per_warp(E);
+  const int nwarps = (tb + 31) / 32;                 // warps that own tokens
+  const int ld = E + 1;                              // padded logit row (no bank conflicts)
+  float* lg = reinterpret_cast<float*>(smem_raw + nwarps * pw);
+  float* bias_sm = lg + static_cast<size_t>(tb) * ld;
+  const int t0 = blockIdx.x * tb;
+  const int nt = min(tb, T - t0);
+
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bias_sm[e] = bias != nullptr ? bias[e] : 0.f;
+  // 1. partial sums of the block's nt x E logits (one contiguous range per slice)
+  const size_t slice = static_cast<size_t>(T) * E;
+  const float* base = part + static_cast<size_t>(t0) * E;
+  const int n = nt * E;
+  if ((E & 3) == 0) {
+    const int n4 = n / 4;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kRowsThreads) {
+      float4 acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+      for (int ks = 0; ks < KS; ++ks) {
+        const float4* src = reinterpret_cast<const float4*>(base + ks * slice);
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[u] = (i0 + u * kRowsThreads < n4) ? __ldg(src + i0 + u * kRowsThreads) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc[u].x += v[u].x;
+          acc[u].y += v[u].y;
+          acc[u].z += v[u].z;
+          acc[u].w += v[u].w;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i4 = i0 + u * kRowsThreads;
+        if (i4 < n4) {
+          const int i = 4 * i4, r = i / E, e = i - r * E;  // E % 4 == 0: the 4 stay in one row
+          float* d = lg + r * ld + e;
+          d[0] = acc[u].x;
+          d[1] = acc[u].y;
+          d[2] = acc[u].z;
+          d[3] = acc[u].w;
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += kRowsThreads) {
+      float l = 0.f;
+      for (int ks = 0; ks < KS; ++ks) l += __ldg(base + ks * slice + i);
+      const int r = i / E;
+      lg[r * ld + (i - r * E)] = l;
+    }
+  }
+  __syncthreads();
+  if (warp >= nwarps) return;
+
+  // 2. per-thread selection of the NS largest biased scores
+  const int r = threadIdx.x;  // token row within the block
+  const bool has = r < nt;
+  bool flagged = false;
+  if (has) {
+    float val[NS], sv[NS];
+    int id[NS];
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      val[j] = -INFINITY;
+      sv[j] = 0.f;
+      id[j] = 0x7fffffff;
+    }
+    const float* row = lg + r * ld;
+    for (int e = 0; e < E; ++e) {
+      const float s = 1.f / (1.f + expf(-row[e]));
+      const float b = s + bias_sm[e];
+      if (b > val[NS - 1]) keep_top<NS>(val, sv, id, b, s, e);
+    }
+    // 3. certain order unless two adjacent values among the top k+1 are near
+#pragma unroll
+    for (int j = 0; j + 1 < NS; ++j)
+      if (j < k && val[j] - val[j + 1] < tau) flagged = true;
+    if (!flagged) {
+      float wsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < NS; ++j)
+        if (j < k) wsum += sv[j];
+      const size_t o = static_cast<size_t>(t0 + r) * k;
+#pragma unroll
+      for (int j = 0; j < NS; ++j)
+        if (j < k) {
+          ids_out[o + j] = id[j];
+          w_out[o + j] = renorm ? (sv[j] / wsum) * alpha : sv[j] * alpha;
+        }
+    }
+  }
+  uint32_t todo = __ballot_sync(0xffffffffu, flagged);
+  if (todo == 0u) return;
+  const WarpArea w = warp_area(smem_raw + warp * pw, E);
+  while (todo != 0u) {
+    const int f = __ffs(todo) - 1;
+    todo &= todo - 1u;
+    const int rr = warp * 32 + f;
+    const int t = t0 + rr;
+    for (int e = lane; e < E; e += 32) {
+      const float s = 1.f / (1.f + expf(-lg[rr * ld + e]));
+      w.s[e] = s;
+      w.b[e] = s + bias_sm[e];
+    }
+    __syncwarp();
+    const int nn = warp_extract(w, E, k, tau, lane);
+    warp_rerank(w, nn, x + static_cast<size_t>(t) * H, wr, bias, H, k, tau, false, lane);
+    warp_emit(w, k, alpha, renorm, lane, ids_out + static_cast<size_t>(t) * k, w_out + static_cast<size_t>(t) * k);
+    __syncwarp();
+  }
+}
+
+// Tokens per block of the row kernel: its logits take about 16 KB of shared
+// memory (a multiple of 8 tokens, at most one per thread), so a layer of a
+// few thousand tokens still spreads over many SMs.
+int rows_tokens_per_block(int E) { return std::max(8, std::min(kRowsThreads, (4096 / std::max(E, 1)) / 8 * 8)); }
+
+size_t rows_smem(int E, int tb) {
+  const int nwarps = (tb + 31) / 32;
+  return static_cast<size_t>(nwarps) * topk_smem_per_warp(E) +
+         (static_cast<size_t>(tb) * (E + 1) + static_cast<size_t>(E)) * sizeof(float);
 }
 
 }  // namespace
 
-RouterPlan router_plan(int T, int E, int H) {
+RouterPlan router_plan(int T, int E, int H, int num_sms) {
   RouterPlan p;
   const int n_mma = router_mma_n(E);
   const int tiles0 = ((T + 127) / 128) * ((E + n_mma - 1) / n_mma);
-  const int total_kb = 3 * ((H + 63) / 64);
-  int ks = (148 + tiles0 - 1) / tiles0;          // about one wave of CTAs
-  ks = std::min(ks, std::max(1, total_kb / 4));  // at least 4 k-blocks per split
+  const int steps = splitk_steps(H, 3, n_mma, T);
+  int ks = std::max(1, num_sms / tiles0);        // at most one wave of CTAs
+  ks = std::min(ks, std::max(1, steps / 4));     // at least 4 K steps per split
   ks = std::min(ks, std::max(1, kRouterPartialRows / std::max(T, 1)));
   ks = std::min(ks, 32);  // the top-k kernel adds every slice: keep its reads short
-  p.ks = router_actual_splits(H, std::max(ks, 1));
+  p.ks = router_actual_splits(T, E, H, std::max(ks, 1));
   return p;
 }
 
@@ -322,12 +507,12 @@ size_t router_partial_floats(int Tmax, int E) {
   return static_cast<size_t>(E) * static_cast<size_t>(std::max(Tmax + 64, kRouterPartialRows));
 }
 
-size_t router_topk_smem(int E) { return static_cast<size_t>(kTopkWarps) * topk_smem_per_warp(E); }
+size_t router_topk_smem(int E) { return topk_smem_per_warp(E); }
 
 cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const void* x, int T, int32_t* ids,
                           float* wts, float* part, void* w_split, int32_t* err, int num_sms, cudaStream_t stream) {
   const int E = cfg.num_experts, H = cfg.hidden, k = cfg.top_k;
-  const RouterPlan p = router_plan(T, E, H);
+  const RouterPlan p = router_plan(T, E, H, num_sms);
   const int n4 = E * H / 4;
   router_split_kernel<<<(n4 + 255) / 256, 256, 0, stream>>>(reinterpret_cast<const float4*>(w.router_w), n4,
                                                              static_cast<uint2*>(w_split));
@@ -335,16 +520,32 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
   if (err_c != cudaSuccess) return err_c;
   err_c = launch_router_gemm(x, T, H, w_split, E, p.ks, part, err, num_sms, stream);
   if (err_c != cudaSuccess) return err_c;
-  const size_t smem = router_topk_smem(E);
-  err_c = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_kernel),
-                           static_cast<int>(router_topk_smem(MOE_MAX_EXPERTS)));
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (T < num_sms * kTopkWarps) {
+    // few tokens: one token per block, so 256 threads read its partial sums
+    err_c = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_coop_kernel),
+                             static_cast<int>(router_topk_smem(MOE_MAX_EXPERTS)));
+    if (err_c != cudaSuccess) return err_c;
+    router_topk_coop_kernel<<<T, kTopkWarps * 32, router_topk_smem(E), stream>>>(
+        part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
+        kRouterTieTau, ids, wts);
+    return cudaGetLastError();
+  }
+  const int tb = rows_tokens_per_block(E);
+  const size_t smem = rows_smem(E, tb);
+  const unsigned grid = static_cast<unsigned>((T + tb - 1) / tb);
+  const void* fn = k < 8 ? reinterpret_cast<const void*>(router_topk_rows_kernel<8>)
+                         : reinterpret_cast<const void*>(router_topk_rows_kernel<MOE_MAX_TOP_K + 1>);
+  err_c = ensure_smem_attr(fn, static_cast<int>(rows_smem(MOE_MAX_EXPERTS, rows_tokens_per_block(MOE_MAX_EXPERTS))));
   if (err_c != cudaSuccess) return err_c;
-  // few tokens: one token per block so the partial sums are read by 256
-  // threads at once; many tokens: one token per warp
-  const int tpb = T >= 148 * kTopkWarps ? kTopkWarps : 1;
-  router_topk_kernel<<<(T + tpb - 1) / tpb, kTopkWarps * 32, smem, stream>>>(
-      part, p.ks, static_cast<const __nv_bfloat16*>(x), w.router_w, w.correction_bias, T, E, H, k,
-      cfg.routed_scaling_factor, cfg.renormalize, kRouterTieTau, tpb, ids, wts);
+  if (k < 8)
+    router_topk_rows_kernel<8><<<grid, kRowsThreads, smem, stream>>>(
+        part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
+        kRouterTieTau, tb, ids, wts);
+  else
+    router_topk_rows_kernel<MOE_MAX_TOP_K + 1><<<grid, kRowsThreads, smem, stream>>>(
+        part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
+        kRouterTieTau, tb, ids, wts);
   return cudaGetLastError();
 }
 

@@ -15,11 +15,16 @@
 // Tile: 128 A rows x n_mma (<= 256) columns, K step 64 (one 128-byte
 // swizzle atom); rows past the end of A are zero-filled by TMA and never
 // stored.  Warps 0-3: epilogue (TMEM -> registers -> global fp32), warp 4:
-// TMA producer, warp 5: TMEM owner + MMA issuer.  A 4-stage smem ring feeds
-// the MMA; two TMEM accumulators let the epilogue of tile i overlap the MMAs
-// of tile i+1.  Every mbarrier wait is bounded; on timeout the kernel records
-// MOE_ERR_DEVICE_TIMEOUT in the workspace error word, drains its own
-// in-flight copies and MMAs, frees TMEM and returns.
+// TMA producer, warp 5: TMEM owner + MMA issuer.  A shared-memory ring of as
+// many stages as fit (up to 8) feeds the MMA: with a narrow B (the router's
+// E columns) or few A rows (a handful of tokens) a stage is small, and what
+// bounds the copy rate is the bytes in flight per SM, not the bytes per
+// stage.  When the B slices are narrow (n_mma <= 128) one stage holds the A
+// tile and the same K range of every B slice, so A is copied once for all
+// passes instead of once per pass.  Two TMEM accumulators let the epilogue
+// of tile i overlap the MMAs of tile i+1.  Every mbarrier wait is bounded; on
+// timeout the kernel records MOE_ERR_DEVICE_TIMEOUT in the workspace error
+// word, drains its own in-flight copies and MMAs, frees TMEM and returns.
 #include <cstring>
 
 #include "moe_internal.h"
@@ -31,10 +36,9 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int MMA_N = 256;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB
-constexpr int B_BYTES = MMA_N * BK * 2;    // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int kMaxStages = 8;
+constexpr int kRingBytes = 224 * 1024;     // shared-memory ring budget
+constexpr int kMaxInnerStageBytes = 64 * 1024;  // B slices share a stage only while 3 stages fit
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -49,8 +53,13 @@ struct alignas(64) SplitKParams {
   int32_t k_blocks;           // k-blocks of one pass over K
   int32_t parts;              // passes over K (slices of B)
   int32_t k_splits;           // tiles split along the (parts x k-blocks) range
-  int32_t kb_per_split;
+  int32_t kb_per_split;       // K steps per split
   int32_t n_tiles;            // output-column tiles x k_splits
+  int32_t stages;             // ring stages (<= kMaxStages)
+  int32_t stage_bytes;        // A region + B slices of one stage (multiple of 1024)
+  int32_t a_bytes;            // A region of a stage (multiple of 1024)
+  int32_t b_bytes;            // one B slice of a stage: n_mma rows x 128 bytes
+  int32_t parts_per_stage;    // 1: one B slice per K step; parts: every slice
   uint32_t idesc;             // MMA instruction descriptor
   int32_t* err;
   int32_t a_box_rows;         // rows per A copy: 128, or fewer when A has fewer rows
@@ -59,8 +68,8 @@ struct alignas(64) SplitKParams {
 };
 
 struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t mma_done;
@@ -68,8 +77,8 @@ struct SmemCtl {
   int32_t abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + sizeof(SmemCtl);
-static_assert(kSmemBytes <= 232448, "fits the 227 KB opt-in shared memory");
+constexpr size_t kSmemMax = 1024 /*align slack*/ + kRingBytes + sizeof(SmemCtl);
+static_assert(kSmemMax <= 232448, "fits the 227 KB opt-in shared memory");
 
 struct TileInfo {
   int row0;     // first token row of the tile
@@ -91,9 +100,10 @@ __device__ __forceinline__ TileInfo decode_tile(const SplitKParams& P, int t) {
   return ti;
 }
 
-// k-blocks [kb0, kb1) of the (parts x k-blocks) range a tile accumulates.
+// K steps [kb0, kb1) a tile accumulates: of the (parts x k-blocks) range, or
+// of the k-blocks alone when every B slice shares the stage.
 __device__ __forceinline__ void tile_k_range(const SplitKParams& P, const TileInfo& ti, int& kb0, int& kb1) {
-  const int total = P.k_blocks * P.parts;
+  const int total = P.parts_per_stage == 1 ? P.k_blocks * P.parts : P.k_blocks;
   kb0 = ti.split * P.kb_per_split;
   kb1 = min(total, kb0 + P.kb_per_split);
 }
@@ -102,9 +112,8 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
-  unsigned char* smem_a = smem;
-  unsigned char* smem_b = smem + STAGES * A_BYTES;
-  SmemCtl& c = *reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+  const int STAGES = P.stages;
+  SmemCtl& c = *reinterpret_cast<SmemCtl*>(smem + STAGES * P.stage_bytes);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -152,20 +161,24 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         const int ncol0 = ti.nidx * P.n_mma;
         int kb0, kb1;
         tile_k_range(P, ti, kb0, kb1);
-        // A rows past a_box_rows stay stale in shared memory: they only feed
+        // A rows past a_box_rows are not copied: the MMA reads whatever the
+        // stage holds there (the B slices that follow A), which only feeds
         // accumulator rows that are never stored
-        const uint32_t stage_tx = static_cast<uint32_t>((P.a_box_rows + P.n_mma) * BK * 2);
+        const int nps = P.parts_per_stage;
+        const uint32_t stage_tx = static_cast<uint32_t>((P.a_box_rows + nps * P.n_mma) * BK * 2);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.timeout_ns)) {
             fail(1);
             ok = false;
             break;
           }
-          const int part = kb / P.k_blocks;
+          const int part = nps == 1 ? kb / P.k_blocks : 0;
           const int kc = (kb - part * P.k_blocks) * BK;
+          unsigned char* st = smem + stage * P.stage_bytes;
           mbar_arrive_expect_tx(&c.full[stage], stage_tx);
-          tma_load_2d(smem_a + stage * A_BYTES, &P.tma_a, kc, ti.row0, &c.full[stage]);
-          tma_load_3d(smem_b + stage * B_BYTES, &P.tma_b, kc, ncol0, part, &c.full[stage]);
+          tma_load_2d(st, &P.tma_a, kc, ti.row0, &c.full[stage]);
+          for (int q = 0; q < nps; ++q)
+            tma_load_3d(st + P.a_bytes + q * P.b_bytes, &P.tma_b, kc, ncol0, part + q, &c.full[stage]);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -209,13 +222,15 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem_a + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(smem_b + stage * B_BYTES);
+          const uint32_t a_addr = smem_u32(smem + stage * P.stage_bytes);
+          for (int q = 0; q < P.parts_per_stage; ++q) {
+            const uint32_t b_addr = a_addr + static_cast<uint32_t>(P.a_bytes + q * P.b_bytes);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
-            const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
+              umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || q > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&c.empty[stage]);
           if (++stage == STAGES) {
@@ -316,6 +331,26 @@ bool encode_b(CUtensorMap* m, const void* base, int slices, int N, int K, int bo
   return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Ring geometry: A region of a_box_rows rows (rounded up to whole 8-row
+// swizzle atoms), B slices of n_mma rows; all B slices in one stage when
+// that keeps at least three stages, else one slice per stage.  Stage sizes
+// are multiples of 1024 bytes (whole swizzle atoms at aligned addresses).
+void set_geometry(SplitKParams& P, int n_mma, int parts, int a_box_rows) {
+  P.a_bytes = (a_box_rows * BK * 2 + 1023) / 1024 * 1024;
+  P.b_bytes = n_mma * BK * 2;
+  const int inner = P.a_bytes + parts * P.b_bytes;
+  P.parts_per_stage = (parts > 1 && inner <= kMaxInnerStageBytes) ? parts : 1;
+  // the M = 128 MMA reads 128 rows of A (16 KB) from the start of a stage
+  // whatever a_box_rows is: a stage is never shorter, so that read stays
+  // inside the ring
+  P.stage_bytes = std::max(P.a_bytes + P.parts_per_stage * P.b_bytes, BM * BK * 2);
+  P.stages = std::min(kMaxStages, kRingBytes / P.stage_bytes);
+}
+
+size_t smem_bytes(const SplitKParams& P) {
+  return 1024 + static_cast<size_t>(P.stages) * P.stage_bytes + sizeof(SmemCtl);
+}
+
 }  // namespace
 
 cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, int parts, int N, int n_mma,
@@ -335,7 +370,8 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   P.n_mma = n_mma;
   P.k_blocks = (K + BK - 1) / BK;
   P.parts = parts;
-  const int total = parts * P.k_blocks;
+  set_geometry(P, n_mma, parts, a_box);
+  const int total = P.parts_per_stage == 1 ? parts * P.k_blocks : P.k_blocks;
   const int kbps = (total + k_splits - 1) / k_splits;
   P.kb_per_split = kbps;
   P.k_splits = (total + kbps - 1) / kbps;
@@ -343,10 +379,10 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   P.idesc = umma_idesc_bf16(BM, n_mma);
   P.err = err;
   P.timeout_ns = kTimeoutNs;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemBytes));
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemMax));
   if (e != cudaSuccess) return e;
   const int tiles = ((rows + BM - 1) / BM) * P.n_tiles;
-  splitk_gemm_kernel<<<std::min(num_sms, tiles), THREADS, kSmemBytes, stream>>>(P);
+  splitk_gemm_kernel<<<std::min(num_sms, tiles), THREADS, smem_bytes(P), stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -371,6 +407,7 @@ cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStre
   P.n_mma = 16;
   P.k_blocks = 1;
   P.parts = 1;
+  set_geometry(P, 16, 1, BM);
   P.kb_per_split = 1;
   P.k_splits = 1;
   P.n_tiles = 1;
@@ -378,14 +415,22 @@ cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStre
   P.err = err;
   P.timeout_ns = 20000000ull;
   P.test_withhold = 1;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemBytes));
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemMax));
   if (e != cudaSuccess) return e;
-  splitk_gemm_kernel<<<1, THREADS, kSmemBytes, stream>>>(P);
+  splitk_gemm_kernel<<<1, THREADS, smem_bytes(P), stream>>>(P);
   return cudaGetLastError();
 }
 
-int splitk_actual_splits(int K, int parts, int k_splits) {
-  const int total = parts * ((K + BK - 1) / BK);
+int splitk_steps(int K, int parts, int n_mma, int rows) {
+  SplitKParams P;
+  memset(&P, 0, sizeof(P));
+  set_geometry(P, n_mma, parts, rows < BM ? std::max(8, (rows + 7) / 8 * 8) : BM);
+  const int kb = (K + BK - 1) / BK;
+  return P.parts_per_stage == 1 ? parts * kb : kb;
+}
+
+int splitk_actual_splits(int K, int parts, int n_mma, int rows, int k_splits) {
+  const int total = splitk_steps(K, parts, n_mma, rows);
   const int kbps = (total + k_splits - 1) / k_splits;
   return (total + kbps - 1) / kbps;
 }
@@ -395,6 +440,8 @@ cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split,
   return launch_splitk_gemm(x, T, H, w_split, 3, E, router_mma_n(E), k_splits, part, err, num_sms, stream);
 }
 
-int router_actual_splits(int H, int k_splits) { return splitk_actual_splits(H, 3, k_splits); }
+int router_actual_splits(int T, int E, int H, int k_splits) {
+  return splitk_actual_splits(H, 3, router_mma_n(E), T, k_splits);
+}
 
 }  // namespace moe

@@ -64,6 +64,10 @@ EDGE = {
                                     swiglu_limit=255.0, x_scale=50.0, w4a16=True),
     "w4a16_prefill_wide_limit": LayerConfig("w4a16_prefill_wide_limit", T=300, H=256, E=4, k=2, I=256,
                                             I_s=128, swiglu_limit=255.0, x_scale=50.0, w4a16=True),
+    # enough tokens for the row-block top-k kernel: E not a multiple of 4
+    # (scalar partial sums), and k >= 8 (17 kept values per thread)
+    "rows_e5": LayerConfig("rows_e5", T=1300, H=128, E=5, k=3, I=64, I_s=32, alpha=1.5, renorm=True),
+    "rows_k10": LayerConfig("rows_k10", T=1250, H=256, E=40, k=10, I=64, I_s=0),
     "shared_small_t32": LayerConfig("shared_small_t32", T=32, H=256, E=4, k=2, I=64, I_s=96, alpha=2.5,
                                     renorm=True),
     "shared_tc_t33": LayerConfig("shared_tc_t33", T=33, H=256, E=4, k=2, I=64, I_s=96),
@@ -92,14 +96,24 @@ def _tied_router_inputs():
     return inp
 
 
+def _tied_router_rows_inputs():
+    # enough tokens for the row-block top-k kernel (one token per thread),
+    # whose exact ties must fall back to the warp path and its fp64 re-order
+    cfg = LayerConfig("tied_router_rows", T=1400, H=256, E=8, k=3, I=64, I_s=0, bias_kind="zero")
+    inp = moe_inputs.make_layer(cfg, seed=6)
+    inp.router_w[4:8] = inp.router_w[0:4]
+    return inp
+
+
 def _all_small_inputs():
     out = {n: _edge_inputs(n) for n in EDGE}
     out["hot_expert"] = _hot_expert_inputs()
     out["tied_router"] = _tied_router_inputs()
+    out["tied_router_rows"] = _tied_router_rows_inputs()
     return out
 
 
-SMALL = sorted(list(EDGE) + ["hot_expert", "tied_router"])
+SMALL = sorted(list(EDGE) + ["hot_expert", "tied_router", "tied_router_rows"])
 
 
 @pytest.fixture(scope="module")
@@ -172,6 +186,7 @@ def test_tile_queues_are_left_at_zero(small_inputs, name):
         header = layer.ws[:256].view(torch.int32).cpu()
         assert header[0].item() == 0, "device error word set"
         assert torch.count_nonzero(header[2:10]).item() == 0, f"tile queue words {header[2:10].tolist()}"
+        assert header[10].item() == 0, "permute ticket counter left non-zero"
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
@@ -201,8 +216,9 @@ def test_forward_replays_from_a_cuda_graph(small_inputs, name):
     del graph
 
 
-def test_tied_router_prefers_lower_id(small_inputs):
-    inp = small_inputs["tied_router"]
+@pytest.mark.parametrize("name", ["tied_router", "tied_router_rows"])
+def test_tied_router_prefers_lower_id(small_inputs, name):
+    inp = small_inputs[name]
     layer = gpu_layer(inp)
     st = run_stages(layer, inp.x.cuda())
     sel = oracle.select_topk(oracle.router_logits(inp.x, inp.router_w), inp.correction_bias, inp.cfg.k, 1.0,
