@@ -276,6 +276,26 @@ MOE_API moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t*
 #define MOE_SELFTEST_SCRATCH_BYTES 65536
 MOE_API moe_status moe_selftest_device_timeout(void* scratch, size_t scratch_bytes, moe_stream_t stream);
 
+/* Test hook for the timeout paths of the grouped GEMMs that run on CTA
+ * pairs; the pages have no counterpart.  Zeroes `scratch` (as above; its
+ * first 256 bytes are laid out like a workspace header) and launches one
+ * pair (two CTAs on two SMs) of
+ *   MOE_SELFTEST_PAIR_BF16: the bf16 grouped gate/up kernel, or
+ *   MOE_SELFTEST_PAIR_INT4: the int4 (W4A16 prefill) grouped gate/up kernel,
+ * on one tiny tile of zero operands held in scratch, with the signal that
+ * the tile's accumulator is complete never sent to the epilogue and every
+ * wait on another role limited to 20 ms.  Both CTAs' epilogue waits run
+ * out; the kernel records MOE_ERR_DEVICE_TIMEOUT in scratch's error word,
+ * every other role finishes, the copies and MMAs drain, the pair resets
+ * its tile-queue words in the header to zero and frees its tensor memory,
+ * and the context stays usable.  Read the result with
+ * moe_read_device_error(scratch, ...).  Returns MOE_OK once the launch is
+ * enqueued; MOE_ERR_INVALID_ARG for another `kernel`. */
+#define MOE_SELFTEST_PAIR_BF16 0
+#define MOE_SELFTEST_PAIR_INT4 1
+MOE_API moe_status moe_selftest_pair_timeout(void* scratch, size_t scratch_bytes, int32_t kernel,
+                                             moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,10 +32,12 @@ MOE_INT4_MAX_SWIGLU_LIMIT = 255.0
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",
     "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward",
-    "moe_read_device_error", "moe_permute_no_alloc", "moe_selftest_device_timeout",
+    "moe_read_device_error", "moe_permute_no_alloc", "moe_selftest_device_timeout", "moe_selftest_pair_timeout",
 )
 MOE_NO_ALLOC_MAX_ROWS = 131072
 MOE_SELFTEST_SCRATCH_BYTES = 65536
+MOE_SELFTEST_PAIR_BF16 = 0
+MOE_SELFTEST_PAIR_INT4 = 1
 
 
 class MoEError(RuntimeError):
@@ -98,6 +100,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_forward": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, SZ, P]),
         "moe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
         "moe_selftest_device_timeout": (ctypes.c_int, [P, SZ, P]),
+        "moe_selftest_pair_timeout": (ctypes.c_int, [P, SZ, I32, P]),
         "moe_permute_no_alloc": (ctypes.c_int, [CFG, P, P, P, I32, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -220,6 +223,14 @@ def moe_selftest_device_timeout(scratch, stream=None):
     moe_read_device_error(scratch))."""
     _check(load_library().moe_selftest_device_timeout(_ptr(scratch), scratch.numel() * scratch.element_size(),
                                                       _stream(stream)), "moe_selftest_device_timeout")
+
+
+def moe_selftest_pair_timeout(scratch, kernel, stream=None):
+    """Test hook: force the timeout path of a CTA-pair grouped GEMM
+    (MOE_SELFTEST_PAIR_BF16 or MOE_SELFTEST_PAIR_INT4) on a tiny tile; read
+    the error with moe_read_device_error(scratch)."""
+    _check(load_library().moe_selftest_pair_timeout(_ptr(scratch), scratch.numel() * scratch.element_size(),
+                                                    int(kernel), _stream(stream)), "moe_selftest_pair_timeout")
 
 
 def status_strings():

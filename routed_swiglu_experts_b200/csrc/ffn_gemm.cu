@@ -82,6 +82,8 @@ struct alignas(64) PairParams {
   float limit;
   int32_t* err;
   int32_t* queue;             // {next tile, pairs retired}: zero at launch, left zero at exit
+  uint64_t wait_ns;           // limit of every wait on another role's progress
+  int32_t test_withhold;      // test hook: never signal the first tile's accumulator to the epilogue
 };
 
 struct Ctl {
@@ -260,7 +262,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // asks first, so pairs that drew cheap (ragged) tiles take more.
         int t;
         if (leader) {
-          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, P.wait_ns)) {
             fail(35);
             break;
           }
@@ -272,7 +274,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
           mbar_arrive(&c.tq_full[q]);
         } else {
-          if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, P.wait_ns)) {
             fail(36);
             break;
           }
@@ -293,7 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int nstage = (nkb + KCH - 1) / KCH;  // the last stage of an odd count holds one chunk
         const int kpre = nstage > 2 ? nstage - 2 : 0;
         for (int st = 0; st < nstage; ++st) {
-          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns)) {
             fail(31);
             ok = false;
             break;
@@ -347,11 +349,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader && lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
+      bool ok = true, first = true;
       int q = 0;
       uint32_t qph = 0;
       for (;;) {
-        if (!mbar_wait_bounded(&c.tq_full[q], qph, abort_flag, kTimeoutNs)) {
+        if (!mbar_wait_bounded(&c.tq_full[q], qph, abort_flag, P.wait_ns)) {
           fail(37);
           break;
         }
@@ -365,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const Tile ti = decode(P, c, t);
         const int p = ti.p;
         const uint32_t idesc = umma_idesc_bf16(2 * ROWS, ti.nmma);
-        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, P.wait_ns)) {
           fail(32);
           break;
         }
@@ -374,7 +376,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int nkb = P.k_blocks[p];
         const int nstage = (nkb + KCH - 1) / KCH;
         for (int st = 0; st < nstage; ++st) {
-          if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, P.wait_ns)) {
             fail(33);
             ok = false;
             break;
@@ -400,7 +402,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair(&c.tmem_full[acc]);
+        if (!(P.test_withhold && first)) umma_commit_pair(&c.tmem_full[acc]);
+        first = false;
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
@@ -420,7 +423,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     int q = 0;
     uint32_t qph = 0;
     for (;;) {
-      const bool gotq = mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, kTimeoutNs);
+      const bool gotq = mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, P.wait_ns);
       if (!named_barrier_and(1, 128, gotq)) {
         if (lane == 0 && !gotq) fail(40);
         break;
@@ -436,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const Tile ti = decode(P, c, t);
       const int p = ti.p;
       const int N = P.n_out[p];
-      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
+      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, P.wait_ns);
       // all four warps leave together: the gate/up exchange below uses named barriers
       if (!named_barrier_and(1, 128, got)) {
         if (lane == 0 && !got) fail(34);
@@ -622,6 +625,7 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
   P.limit = limit;
   P.err = err;
   P.queue = queue;
+  P.wait_ns = kTimeoutNs;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<KIND>), static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   int grid = std::max(2, num_sms / 2 * 2);
@@ -632,6 +636,41 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
 }
 
 }  // namespace
+
+// Test hook: one tiny gate/up problem (16 tokens, 64 features, K = 64; zero
+// operands in `scratch`) on one CTA pair whose first (only) accumulator is
+// never signalled to the epilogue, with every wait on another role limited to
+// 20 ms.  Both CTAs' epilogue waits run out and record
+// MOE_ERR_DEVICE_TIMEOUT (detail 34); the producer, the MMA issuer and the
+// pair's final cluster barrier finish on their normal paths (the copies and
+// MMAs drained, the tile queue reset by the retiring pair, TMEM freed).
+cudaError_t launch_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* queue, cudaStream_t stream) {
+  unsigned char* base = static_cast<unsigned char*>(scratch);
+  void* x = base + 1024;   // bf16 [16, 64]
+  void* w = base + 4096;   // bf16 [1, 2 x 64, 64]: gate rows, then up rows
+  void* h = base + 20480;  // bf16 [16, 64]
+  PairParams P;
+  memset(&P, 0, sizeof(P));
+  if (!encode_x(&P.tma_x[0], x, 16, 64) || !encode_w_gu(&P.tma_w[0], w, 1, 64, 64)) return cudaErrorInvalidValue;
+  P.offsets[0] = nullptr;
+  P.out[0] = static_cast<__nv_bfloat16*>(h);
+  P.groups[0] = 1;
+  P.rows[0] = 16;
+  P.n_out[0] = 64;
+  P.k_blocks[0] = 1;
+  P.f_tiles[0] = 1;
+  P.nprob = 1;
+  P.limit = 7.f;
+  P.err = err;
+  P.queue = queue;
+  P.wait_ns = 20000000ull;
+  P.test_withhold = 1;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<Kind::GateUp>),
+                                   static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  ffn_pair_kernel<Kind::GateUp><<<2, THREADS, kSmem, stream>>>(P);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
                                int32_t* queue, int num_sms, cudaStream_t stream) {

@@ -69,6 +69,8 @@ struct alignas(64) Int4Params {
   float limit;
   int32_t* err;
   int32_t* queue;             // {next tile, pairs retired}: zero at launch, left zero at exit
+  uint64_t wait_ns;           // limit of every wait on another role's progress
+  int32_t test_withhold;      // test hook: never signal the first tile's accumulator to the epilogue
 };
 
 struct Ctl {
@@ -147,8 +149,9 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
 
 // Reader side of the tile-id ring: wait until slot q holds the next id (it
 // may have been stored by the other CTA of the pair: cluster-scope acquire).
-__device__ __forceinline__ bool wait_tile(Ctl& c, int q, uint32_t qph, volatile int32_t* abort, int& t) {
-  if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort, kTimeoutNs)) return false;
+__device__ __forceinline__ bool wait_tile(Ctl& c, int q, uint32_t qph, volatile int32_t* abort, uint64_t limit_ns,
+                                          int& t) {
+  if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort, limit_ns)) return false;
   t = c.tq[q];
   return true;
 }
@@ -269,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // queue and publishes it to every role of both CTAs.
         int t;
         if (leader) {
-          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, P.wait_ns)) {
             fail(50);
             break;
           }
@@ -281,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
           mbar_arrive(&c.tq_full[q]);
         } else {
-          if (!wait_tile(c, q, qph, abort_flag, t)) {
+          if (!wait_tile(c, q, qph, abort_flag, P.wait_ns, t)) {
             fail(51);
             break;
           }
@@ -293,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
         const int kpre = P.k_blocks > 3 ? P.k_blocks - 3 : 0;  // fetch the next id a few copies early
         for (int kb = 0; kb < P.k_blocks; ++kb) {
-          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns)) {
             fail(41);
             ok = false;
             break;
@@ -334,12 +337,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (leader && lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
+      bool ok = true, first = true;
       int q = 0;
       uint32_t qph = 0;
       for (;;) {
         int t;
-        if (!wait_tile(c, q, qph, abort_flag, t)) {
+        if (!wait_tile(c, q, qph, abort_flag, P.wait_ns, t)) {
           fail(52);
           break;
         }
@@ -348,15 +351,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const uint32_t idesc = umma_idesc_f16(2 * ROWS, ti.nmma);
-        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+        if (!mbar_wait_bounded(&c.tmem_empty[acc], acc_phase ^ 1u, abort_flag, P.wait_ns)) {
           fail(42);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         for (int kb = 0; kb < P.k_blocks; ++kb) {
-          if (!mbar_wait_bounded(&c.tok_full[stage], phase, abort_flag, kTimeoutNs) ||
-              !mbar_wait_bounded(&c.full[stage], phase, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.tok_full[stage], phase, abort_flag, P.wait_ns) ||
+              !mbar_wait_bounded(&c.full[stage], phase, abort_flag, P.wait_ns)) {
             fail(43);
             ok = false;
             break;
@@ -375,7 +378,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair(&c.tmem_full[acc]);
+        if (!(P.test_withhold && first)) umma_commit_pair(&c.tmem_full[acc]);
+        first = false;
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
@@ -396,7 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t qph = 0;
       for (;;) {
         int t;
-        if (!wait_tile(c, q, qph, abort_flag, t)) {
+        if (!wait_tile(c, q, qph, abort_flag, P.wait_ns, t)) {
           fail(53);
           break;
         }
@@ -405,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (t < 0) break;
         const Tile ti = decode(P, c, t);
         for (int cb = 0; cb < ncb; ++cb) {
-          if (!mbar_wait_bounded(&c.code_empty[cs], cphase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&c.code_empty[cs], cphase ^ 1u, abort_flag, P.wait_ns)) {
             fail(46);
             ok = false;
             break;
@@ -451,7 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t qph = 0;
     for (;;) {
       int t = -1;
-      const bool gotq = wait_tile(c, q, qph, abort_flag, t);
+      const bool gotq = wait_tile(c, q, qph, abort_flag, P.wait_ns, t);
       if (!__all_sync(0xffffffffu, gotq)) {
         if (lane == 0) fail(54);
         break;
@@ -500,8 +504,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t s2_16 = *reinterpret_cast<const uint32_t*>(&s16h);
         // codes landed (first K step of a copy), and the MMAs have released this A stage
         const int sub = kb % CKB;
-        const bool got = (sub != 0 || mbar_wait_bounded(&c.code_full[cs], cphase, abort_flag, kTimeoutNs)) &&
-                         mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, kTimeoutNs);
+        const bool got = (sub != 0 || mbar_wait_bounded(&c.code_full[cs], cphase, abort_flag, P.wait_ns)) &&
+                         mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns);
         if (!__all_sync(0xffffffffu, got)) {
           if (lane == 0) fail(45);
           ok = false;
@@ -545,7 +549,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t qph = 0;
     for (;;) {
       int t = -1;
-      const bool gotq = wait_tile(c, q, qph, abort_flag, t);
+      const bool gotq = wait_tile(c, q, qph, abort_flag, P.wait_ns, t);
       if (!named_barrier_and(1, 128, gotq)) {
         if (lane == 0 && !gotq) fail(55);
         break;
@@ -556,7 +560,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (t < 0) break;
       const Tile ti = decode(P, c, t);
       const int N = P.n_out;
-      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, kTimeoutNs);
+      const bool got = mbar_wait_bounded(&c.tmem_full[acc], acc_phase, abort_flag, P.wait_ns);
       if (!named_barrier_and(1, 128, got)) {
         if (lane == 0 && !got) fail(44);
         break;
@@ -748,6 +752,7 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
   P.limit = limit;
   P.err = err;
   P.queue = queue;
+  P.wait_ns = kTimeoutNs;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<KIND>), static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   int grid = std::max(2, num_sms / 2 * 2);
@@ -758,6 +763,47 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
 }
 
 }  // namespace
+
+// Test hook: one tiny int4 gate/up problem (16 tokens, 64 features, K = 256;
+// zero codes, scales and tokens in `scratch`, one expert of 16 rows) on one
+// CTA pair whose first (only) accumulator is never signalled to the
+// epilogue, with every wait on another role limited to 20 ms.  Both CTAs'
+// epilogue waits run out and record MOE_ERR_DEVICE_TIMEOUT (detail 44); the
+// token and code producers, the dequantisation warps, the MMA issuer and the
+// pair's final cluster barrier finish on their normal paths.
+cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* queue, cudaStream_t stream) {
+  static const int32_t kOffsets[2] = {0, 16};
+  unsigned char* base = static_cast<unsigned char*>(scratch);
+  void* tokens16 = base + 1024;                             // fp16 [16, 256]
+  void* q = base + 10240;                                   // uint8 [1, 2 x 64, 128]
+  void* scales = base + 26624;                              // bf16 [1, 2 x 64, 2]
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + 27136);  // [0, 16]
+  void* h16 = base + 28672;                                 // fp16 [16, 64]
+  cudaError_t e = cudaMemcpyAsync(offsets, kOffsets, sizeof(kOffsets), cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return e;
+  Int4Params P;
+  memset(&P, 0, sizeof(P));
+  if (!encode_tokens16(&P.tma_x, tokens16, 16, 256) || !encode_codes_gu(&P.tma_q, q, 1, 64, 256))
+    return cudaErrorInvalidValue;
+  P.offsets = offsets;
+  P.scales = static_cast<const __nv_bfloat16*>(scales);
+  P.out = h16;
+  P.groups = 1;
+  P.rows = 16;
+  P.n_out = 64;
+  P.K = 256;
+  P.k_blocks = 256 / BK;
+  P.f_tiles = 1;
+  P.limit = 7.f;
+  P.err = err;
+  P.queue = queue;
+  P.wait_ns = 20000000ull;
+  P.test_withhold = 1;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<Kind::GateUp>), static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  ffn_int4_pair_kernel<Kind::GateUp><<<2, THREADS, kSmem, stream>>>(P);
+  return cudaGetLastError();
+}
 
 bool int4_prefill_preferred(int rows, int E) { return rows >= 32 * E; }
 

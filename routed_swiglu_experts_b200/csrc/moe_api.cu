@@ -358,6 +358,17 @@ moe_status moe_selftest_device_timeout(void* scratch, size_t scratch_bytes, moe_
   return from_cuda(launch_splitk_timeout_selftest(scratch, err_word(scratch), stream));
 }
 
+moe_status moe_selftest_pair_timeout(void* scratch, size_t scratch_bytes, int32_t kernel, moe_stream_t stream) {
+  if (scratch == nullptr || scratch_bytes < MOE_SELFTEST_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (kernel != MOE_SELFTEST_PAIR_BF16 && kernel != MOE_SELFTEST_PAIR_INT4) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(cudaMemsetAsync(scratch, 0, MOE_SELFTEST_SCRATCH_BYTES, stream));
+  if (kernel == MOE_SELFTEST_PAIR_BF16)
+    return from_cuda(launch_pair_timeout_selftest(scratch, err_word(scratch), tile_queue(scratch, kQueueGateUp), stream));
+  return from_cuda(
+      launch_int4_pair_timeout_selftest(scratch, err_word(scratch), tile_queue(scratch, kQueueInt4GateUp), stream));
+}
+
 moe_status moe_read_device_error(void* ws, moe_stream_t stream, int32_t* code) {
   if (ws == nullptr || code == nullptr) return MOE_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;

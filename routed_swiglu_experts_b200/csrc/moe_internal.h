@@ -43,6 +43,9 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
 int splitk_steps(int K, int parts, int n_mma, int rows);
 int splitk_actual_splits(int K, int parts, int n_mma, int rows, int k_splits);
 cudaError_t launch_splitk_timeout_selftest(void* scratch, int32_t* err, cudaStream_t stream);
+// Test hooks of the CTA-pair kernels' timeout paths (see moe_selftest_pair_timeout).
+cudaError_t launch_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* queue, cudaStream_t stream);
+cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* queue, cudaStream_t stream);
 int router_actual_splits(int T, int E, int H, int k_splits);
 cudaError_t launch_router_gemm(const void* x, int T, int H, const void* w_split, int E, int k_splits, float* part,
                                int32_t* err, int num_sms, cudaStream_t stream);

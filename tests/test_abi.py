@@ -186,3 +186,14 @@ def test_selftest_timeout_argument_checks(lib):
     assert lib.moe_selftest_device_timeout(None, n, None) == _abi.MOE_ERR_WORKSPACE
     assert lib.moe_selftest_device_timeout(FAKE, n - 1, None) == _abi.MOE_ERR_WORKSPACE
     assert lib.moe_selftest_device_timeout(FAKE + 16, n, None) == _abi.MOE_ERR_INVALID_ARG
+
+
+def test_pair_selftest_argument_checks(lib):
+    """The CTA-pair timeout hook validates its scratch and kernel selector
+    before touching the GPU."""
+    n = _abi.MOE_SELFTEST_SCRATCH_BYTES
+    assert lib.moe_selftest_pair_timeout(None, n, _abi.MOE_SELFTEST_PAIR_BF16, None) == _abi.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_pair_timeout(FAKE, n - 1, _abi.MOE_SELFTEST_PAIR_BF16, None) == _abi.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_pair_timeout(FAKE + 16, n, _abi.MOE_SELFTEST_PAIR_INT4, None) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_pair_timeout(FAKE, n, 2, None) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_pair_timeout(FAKE, n, -1, None) == _abi.MOE_ERR_INVALID_ARG
