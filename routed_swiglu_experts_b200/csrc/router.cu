@@ -1,7 +1,7 @@
 // Router: the fp32 logits GEMM runs on the tensor cores (splitk_gemm.cu, three
 // passes over K) on an exact bf16 split of the fp32 weight; here are the split
-// and the sigmoid + biased top-k (per token: one thread when the order is
-// certain, one warp with an fp64 re-rank of near-ties when it is not).
+// and the sigmoid + biased top-k (one warp per token, with an fp64 re-rank
+// of near-ties).
 //
 // "Module glm5next_mlp" §Numerics: sigmoid score; the correction bias steers
 // selection only; the emitted weight is the unbiased score times
@@ -316,44 +316,25 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   warp_emit(w, k, alpha, renorm, lane, ids_out + static_cast<size_t>(t) * k, w_out + static_cast<size_t>(t) * k);
 }
 
-// Many tokens: a block takes `tb` consecutive tokens (one per thread of its
-// first tb threads).
+// Many tokens: a block takes `tb` consecutive tokens.
 //  1. All 256 threads sum the block's K-slice partial logits -- contiguous
-//     rows, 16-byte loads, slices in ascending order -- into shared memory.
-//  2. Each token's thread walks its E experts in id order, s = sigmoid(l),
-//     b = s + bias, keeping the NS largest b (desc, ties to the lower id: an
-//     expert enters only by beating the smallest kept value) in registers.
-//  3. If no two adjacent values among the top k+1 are closer than tau, the
-//     order is certain and the thread emits the k ids and weights.  Otherwise
-//     the token's warp takes it: s and b into the warp's scratch, then the
-//     same extraction, fp64 re-order of near-tie clusters and emission as
-//     the few-token kernel.
+//     rows, 16-byte loads, slices in ascending order -- and write every
+//     token's s = sigmoid(l) and b = s + bias rows to shared memory.
+//  2. Each warp takes every 8th token of the block and runs the same
+//     extraction, fp64 re-order of near-tie clusters and emission as the
+//     few-token kernel, reading that token's rows in place.  With many warps
+//     per SM, each on its own token, the latency of the extraction rounds
+//     and of the occasional fp64 dot products overlaps across tokens.
 constexpr int kRowsThreads = 256;
+constexpr int kRowsWarps = kRowsThreads / 32;
 
-template <int NS>
-__device__ __forceinline__ void keep_top(float (&val)[NS], float (&sv)[NS], int (&id)[NS], float b, float s, int e) {
-  // val is sorted descending; b > val[NS-1]: insert it after every kept value
-  // >= b (those have lower ids), shifting the smaller ones down
-#pragma unroll
-  for (int j = NS - 1; j > 0; --j) {
-    if (val[j - 1] < b) {
-      val[j] = val[j - 1];
-      sv[j] = sv[j - 1];
-      id[j] = id[j - 1];
-    } else if (val[j] < b) {
-      val[j] = b;
-      sv[j] = s;
-      id[j] = e;
-    }
-  }
-  if (val[0] < b) {
-    val[0] = b;
-    sv[0] = s;
-    id[0] = e;
-  }
+// A warp's own scratch in the row kernel: v64[E] (fp64), lv[E], lst[E],
+// res[MOE_MAX_TOP_K]; 16-byte multiple.
+__host__ __device__ inline size_t rows_scratch_per_warp(int E) {
+  return (static_cast<size_t>(E) * (8 + 4 + 4) + MOE_MAX_TOP_K * 4 + 15) / 16 * 16;
 }
 
-template <int NS>
+// dynamic smem: kRowsWarps scratch areas | s rows [tb][E] | b rows [tb][E]
 __global__ void __launch_bounds__(kRowsThreads)
     router_topk_rows_kernel(const float* __restrict__ part, int KS, const __nv_bfloat16* __restrict__ x,
                             const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H, int k,
@@ -361,19 +342,22 @@ __global__ void __launch_bounds__(kRowsThreads)
                             float* __restrict__ w_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const size_t pw = topk_smem_per_warp(E);
-  const int nwarps = (tb + 31) / 32;                 // warps that own tokens
-  const int ld = E + 1;                              // padded logit row (no bank conflicts)
-  float* lg = reinterpret_cast<float*>(smem_raw + nwarps * pw);
-  float* bias_sm = lg + static_cast<size_t>(tb) * ld;
+  const size_t pw = rows_scratch_per_warp(E);
+  float* s_rows = reinterpret_cast<float*>(smem_raw + kRowsWarps * pw);
+  float* b_rows = s_rows + static_cast<size_t>(tb) * E;
   const int t0 = blockIdx.x * tb;
   const int nt = min(tb, T - t0);
 
-  for (int e = threadIdx.x; e < E; e += blockDim.x) bias_sm[e] = bias != nullptr ? bias[e] : 0.f;
   // 1. partial sums of the block's nt x E logits (one contiguous range per slice)
   const size_t slice = static_cast<size_t>(T) * E;
   const float* base = part + static_cast<size_t>(t0) * E;
   const int n = nt * E;
+  auto put = [&](int i, float l) {
+    const int e = i % E;
+    const float sv = 1.f / (1.f + expf(-l));
+    s_rows[i] = sv;
+    b_rows[i] = sv + (bias != nullptr ? __ldg(bias + e) : 0.f);
+  };
   if ((E & 3) == 0) {
     const int n4 = n / 4;
     for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kRowsThreads) {
@@ -399,12 +383,10 @@ __global__ void __launch_bounds__(kRowsThreads)
       for (int u = 0; u < 4; ++u) {
         const int i4 = i0 + u * kRowsThreads;
         if (i4 < n4) {
-          const int i = 4 * i4, r = i / E, e = i - r * E;  // E % 4 == 0: the 4 stay in one row
-          float* d = lg + r * ld + e;
-          d[0] = acc[u].x;
-          d[1] = acc[u].y;
-          d[2] = acc[u].z;
-          d[3] = acc[u].w;
+          put(4 * i4, acc[u].x);
+          put(4 * i4 + 1, acc[u].y);
+          put(4 * i4 + 2, acc[u].z);
+          put(4 * i4 + 3, acc[u].w);
         }
       }
     }
@@ -412,64 +394,22 @@ __global__ void __launch_bounds__(kRowsThreads)
     for (int i = threadIdx.x; i < n; i += kRowsThreads) {
       float l = 0.f;
       for (int ks = 0; ks < KS; ++ks) l += __ldg(base + ks * slice + i);
-      const int r = i / E;
-      lg[r * ld + (i - r * E)] = l;
+      put(i, l);
     }
   }
   __syncthreads();
-  if (warp >= nwarps) return;
 
-  // 2. per-thread selection of the NS largest biased scores
-  const int r = threadIdx.x;  // token row within the block
-  const bool has = r < nt;
-  bool flagged = false;
-  if (has) {
-    float val[NS], sv[NS];
-    int id[NS];
-#pragma unroll
-    for (int j = 0; j < NS; ++j) {
-      val[j] = -INFINITY;
-      sv[j] = 0.f;
-      id[j] = 0x7fffffff;
-    }
-    const float* row = lg + r * ld;
-    for (int e = 0; e < E; ++e) {
-      const float s = 1.f / (1.f + expf(-row[e]));
-      const float b = s + bias_sm[e];
-      if (b > val[NS - 1]) keep_top<NS>(val, sv, id, b, s, e);
-    }
-    // 3. certain order unless two adjacent values among the top k+1 are near
-#pragma unroll
-    for (int j = 0; j + 1 < NS; ++j)
-      if (j < k && val[j] - val[j + 1] < tau) flagged = true;
-    if (!flagged) {
-      float wsum = 0.f;
-#pragma unroll
-      for (int j = 0; j < NS; ++j)
-        if (j < k) wsum += sv[j];
-      const size_t o = static_cast<size_t>(t0 + r) * k;
-#pragma unroll
-      for (int j = 0; j < NS; ++j)
-        if (j < k) {
-          ids_out[o + j] = id[j];
-          w_out[o + j] = renorm ? (sv[j] / wsum) * alpha : sv[j] * alpha;
-        }
-    }
-  }
-  uint32_t todo = __ballot_sync(0xffffffffu, flagged);
-  if (todo == 0u) return;
-  const WarpArea w = warp_area(smem_raw + warp * pw, E);
-  while (todo != 0u) {
-    const int f = __ffs(todo) - 1;
-    todo &= todo - 1u;
-    const int rr = warp * 32 + f;
-    const int t = t0 + rr;
-    for (int e = lane; e < E; e += 32) {
-      const float s = 1.f / (1.f + expf(-lg[rr * ld + e]));
-      w.s[e] = s;
-      w.b[e] = s + bias_sm[e];
-    }
-    __syncwarp();
+  // 2. one warp per token
+  unsigned char* mine = smem_raw + warp * pw;
+  WarpArea w;
+  w.v64 = reinterpret_cast<double*>(mine);
+  w.lv = reinterpret_cast<float*>(mine + static_cast<size_t>(E) * 8);
+  w.lst = reinterpret_cast<int*>(w.lv + E);
+  w.res = w.lst + E;
+  for (int r = warp; r < nt; r += kRowsWarps) {
+    const int t = t0 + r;
+    w.s = s_rows + static_cast<size_t>(r) * E;
+    w.b = b_rows + static_cast<size_t>(r) * E;
     const int nn = warp_extract(w, E, k, tau, lane);
     warp_rerank(w, nn, x + static_cast<size_t>(t) * H, wr, bias, H, k, tau, false, lane);
     warp_emit(w, k, alpha, renorm, lane, ids_out + static_cast<size_t>(t) * k, w_out + static_cast<size_t>(t) * k);
@@ -477,15 +417,14 @@ __global__ void __launch_bounds__(kRowsThreads)
   }
 }
 
-// Tokens per block of the row kernel: its logits take about 16 KB of shared
-// memory (a multiple of 8 tokens, at most one per thread), so a layer of a
-// few thousand tokens still spreads over many SMs.
-int rows_tokens_per_block(int E) { return std::max(8, std::min(kRowsThreads, (4096 / std::max(E, 1)) / 8 * 8)); }
+// Tokens per block of the row kernel: 4 per warp when the s and b rows fit
+// in about 64 KB (fewer for large E, at least one per warp).
+int rows_tokens_per_block(int E) {
+  return std::max(kRowsWarps, std::min(4 * kRowsWarps, (8192 / std::max(E, 1)) / kRowsWarps * kRowsWarps));
+}
 
 size_t rows_smem(int E, int tb) {
-  const int nwarps = (tb + 31) / 32;
-  return static_cast<size_t>(nwarps) * topk_smem_per_warp(E) +
-         (static_cast<size_t>(tb) * (E + 1) + static_cast<size_t>(E)) * sizeof(float);
+  return kRowsWarps * rows_scratch_per_warp(E) + 2 * static_cast<size_t>(tb) * E * sizeof(float);
 }
 
 }  // namespace
@@ -532,20 +471,12 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
     return cudaGetLastError();
   }
   const int tb = rows_tokens_per_block(E);
-  const size_t smem = rows_smem(E, tb);
-  const unsigned grid = static_cast<unsigned>((T + tb - 1) / tb);
-  const void* fn = k < 8 ? reinterpret_cast<const void*>(router_topk_rows_kernel<8>)
-                         : reinterpret_cast<const void*>(router_topk_rows_kernel<MOE_MAX_TOP_K + 1>);
-  err_c = ensure_smem_attr(fn, static_cast<int>(rows_smem(MOE_MAX_EXPERTS, rows_tokens_per_block(MOE_MAX_EXPERTS))));
+  err_c = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_rows_kernel),
+                           static_cast<int>(rows_smem(MOE_MAX_EXPERTS, rows_tokens_per_block(MOE_MAX_EXPERTS))));
   if (err_c != cudaSuccess) return err_c;
-  if (k < 8)
-    router_topk_rows_kernel<8><<<grid, kRowsThreads, smem, stream>>>(
-        part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
-        kRouterTieTau, tb, ids, wts);
-  else
-    router_topk_rows_kernel<MOE_MAX_TOP_K + 1><<<grid, kRowsThreads, smem, stream>>>(
-        part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
-        kRouterTieTau, tb, ids, wts);
+  router_topk_rows_kernel<<<static_cast<unsigned>((T + tb - 1) / tb), kRowsThreads, rows_smem(E, tb), stream>>>(
+      part, p.ks, xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor, cfg.renormalize,
+      kRouterTieTau, tb, ids, wts);
   return cudaGetLastError();
 }
 
