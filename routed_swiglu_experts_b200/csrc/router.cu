@@ -152,34 +152,52 @@ __device__ __forceinline__ WarpArea warp_area(unsigned char* base, int E) {
   return w;
 }
 
-// Phase 2 (one warp, w.s and w.b filled): extract experts in (b desc, id
-// asc) order -- the top k+1, and, while the k-th/(k+1)-th boundary is a
-// near-tie, every further expert that continues the run of adjacent gaps
-// below tau.  Returns how many were extracted; res[0..k) = the first k.
+// Phase 2 (one warp, w.s and w.b filled): extract experts in descending
+// order -- the top k+1, and, while the k-th/(k+1)-th boundary is a near-tie,
+// every further expert that continues the run of adjacent gaps below tau.
+// Returns how many were extracted; res[0..k) = the first k.
+//
+// Each round is one warp-wide max (redux.sync) of 32-bit keys: the upper 22
+// bits of the order-preserving integer image of b (sign, exponent and 13
+// mantissa bits) above 10 bits of (1023 - id), so equal prefixes go to the
+// lower id.  Two experts whose b share a 22-bit prefix may come out in either
+// order.  Out of order, they sit next to each other in the extracted list
+// with a negative gap, below tau, so they land in the same near-tie cluster
+// and are re-ordered exactly in phase 3; in order, they are where exact fp32
+// order puts them.  So the selection is the same as extracting by exact
+// fp32 order.
+__device__ __forceinline__ uint32_t order_key(float b, int e) {
+  const uint32_t u = __float_as_uint(b);
+  const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (o & 0xFFFFFC00u) | (1023u - static_cast<uint32_t>(e));
+}
+
 __device__ int warp_extract(const WarpArea& w, int E, int k, float tau, int lane) {
   const int nm = (E + 31) / 32;  // entries per lane: e = lane + 32 m
   uint32_t taken = 0;
+  auto lane_best = [&]() {
+    uint32_t best = 0;
+    for (int m = 0; m < nm; ++m) {
+      const int e = lane + 32 * m;
+      if (e < E && !((taken >> m) & 1u)) best = max(best, order_key(w.b[e], e));
+    }
+    return best;
+  };
+  uint32_t mine = lane_best();
   const int k1 = min(k + 1, E);
   int n = 0;
   while (n < E) {
-    float v = -INFINITY;
-    int id = 0x7fffffff;
-    for (int m = 0; m < nm; ++m) {
-      const int e = lane + 32 * m;
-      if (e < E && !((taken >> m) & 1u)) {
-        const float bv = w.b[e];
-        if (bv > v || (bv == v && e < id)) {
-          v = bv;
-          id = e;
-        }
-      }
-    }
-    warp_argmax(v, id);
+    const uint32_t top = __reduce_max_sync(0xffffffffu, mine);
+    const int id = 1023 - static_cast<int>(top & 1023u);
+    const float v = w.b[id];
     if (n >= k1) {  // past k+1: only while the boundary run continues
       const bool boundary_tie = w.lv[k - 1] - w.lv[k] < tau;
       if (!boundary_tie || !(w.lv[n - 1] - v < tau)) break;
     }
-    if ((id & 31) == lane) taken |= 1u << (id / 32);
+    if ((id & 31) == lane) {
+      taken |= 1u << (id / 32);
+      mine = lane_best();
+    }
     if (lane == 0) {
       w.lst[n] = id;
       w.lv[n] = v;
@@ -320,11 +338,11 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
 //  1. All 256 threads sum the block's K-slice partial logits -- contiguous
 //     rows, 16-byte loads, slices in ascending order -- and write every
 //     token's s = sigmoid(l) and b = s + bias rows to shared memory.
-//  2. Each warp takes every 8th token of the block and runs the same
-//     extraction, fp64 re-order of near-tie clusters and emission as the
-//     few-token kernel, reading that token's rows in place.  With many warps
-//     per SM, each on its own token, the latency of the extraction rounds
-//     and of the occasional fp64 dot products overlaps across tokens.
+//  2. Each warp takes one token of the block and runs the same extraction,
+//     fp64 re-order of near-tie clusters and emission as the few-token
+//     kernel, reading that token's rows in place.  With many warps per SM,
+//     each on its own token, the latency of the extraction rounds and of the
+//     occasional fp64 dot products overlaps across tokens.
 constexpr int kRowsThreads = 256;
 constexpr int kRowsWarps = kRowsThreads / 32;
 
@@ -417,11 +435,9 @@ __global__ void __launch_bounds__(kRowsThreads)
   }
 }
 
-// Tokens per block of the row kernel: 4 per warp when the s and b rows fit
-// in about 64 KB (fewer for large E, at least one per warp).
-int rows_tokens_per_block(int E) {
-  return std::max(kRowsWarps, std::min(4 * kRowsWarps, (8192 / std::max(E, 1)) / kRowsWarps * kRowsWarps));
-}
+// Tokens per block of the row kernel: one per warp, so that every token's
+// latency-bound selection runs on a warp of its own.
+int rows_tokens_per_block(int) { return kRowsWarps; }
 
 size_t rows_smem(int E, int tb) {
   return kRowsWarps * rows_scratch_per_warp(E) + 2 * static_cast<size_t>(tb) * E * sizeof(float);

@@ -21,8 +21,11 @@
 // bounds the copy rate is the bytes in flight per SM, not the bytes per
 // stage.  When the B slices are narrow (n_mma <= 128) one stage holds the A
 // tile and the same K range of every B slice, so A is copied once for all
-// passes instead of once per pass.  Two TMEM accumulators let the epilogue
-// of tile i overlap the MMAs of tile i+1.  Every mbarrier wait is bounded; on
+// passes instead of once per pass, and each slice accumulates into its own
+// TMEM columns (the epilogue adds them, smallest first: for the router's
+// three-way split of an fp32 weight the small parts keep their bits instead
+// of being added into the large running sum).  Two TMEM accumulator sets,
+// where they fit, let the epilogue of tile i overlap the MMAs of tile i+1.  Every mbarrier wait is bounded; on
 // timeout the kernel records MOE_ERR_DEVICE_TIMEOUT in the workspace error
 // word, drains its own in-flight copies and MMAs, frees TMEM and returns.
 #include <cstring>
@@ -35,7 +38,6 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int MMA_N = 256;
 constexpr int kMaxStages = 8;
 constexpr int kRingBytes = 224 * 1024;     // shared-memory ring budget
 constexpr int kMaxInnerStageBytes = 64 * 1024;  // B slices share a stage only while 3 stages fit
@@ -59,7 +61,9 @@ struct alignas(64) SplitKParams {
   int32_t stage_bytes;        // A region + B slices of one stage (multiple of 1024)
   int32_t a_bytes;            // A region of a stage (multiple of 1024)
   int32_t b_bytes;            // one B slice of a stage: n_mma rows x 128 bytes
-  int32_t parts_per_stage;    // 1: one B slice per K step; parts: every slice
+  int32_t parts_per_stage;    // 1: one B slice per K step; parts: every slice, each into its own accumulator
+  int32_t acc_cols;           // TMEM columns of one tile's accumulators (parts_per_stage x n_mma)
+  int32_t acc_bufs;           // accumulator sets in TMEM (2: epilogue overlaps the next tile)
   uint32_t idesc;             // MMA instruction descriptor
   int32_t* err;
   int32_t a_box_rows;         // rows per A copy: 128, or fewer when A has fewer rows
@@ -214,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * MMA_N);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * P.acc_cols);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&c.full[stage], phase, abort_flag, P.timeout_ns)) {
             fail(3);
@@ -225,11 +229,12 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
           const uint32_t a_addr = smem_u32(smem + stage * P.stage_bytes);
           for (int q = 0; q < P.parts_per_stage; ++q) {
             const uint32_t b_addr = a_addr + static_cast<uint32_t>(P.a_bytes + q * P.b_bytes);
+            const uint32_t d_q = d_tmem + static_cast<uint32_t>(q * P.n_mma);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint64_t ad = sw128_kmajor_desc(a_addr + kk * 32);
               const uint64_t bd = sw128_kmajor_desc(b_addr + kk * 32);
-              umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || q > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16(d_q, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(&c.empty[stage]);
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         }
         if (!ok) break;
         if (!(P.test_withhold && t == static_cast<int>(blockIdx.x))) umma_commit(&c.tmem_full[acc]);
-        if (++acc == 2) {
+        if (++acc == P.acc_bufs) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * MMA_N);
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * P.acc_cols);
       const bool row_ok = row_in_tile < ti.nrows;
       const int N = P.n_out;
       const int nch = (P.n_mma + 31) / 32;
@@ -276,8 +281,17 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
       for (int ch = 0; ch < nch; ++ch) {
         uint32_t v[32];
         __syncwarp();
-        tmem_ld32(tbase + ch * 32, v);
+        tmem_ld32(tbase + (P.parts_per_stage - 1) * P.n_mma + ch * 32, v);
         tmem_ld_wait();
+        // per-slice accumulators (narrow B): add them from the last slice
+        // (smallest terms of the router weight's split) to the first
+        for (int q = P.parts_per_stage - 2; q >= 0; --q) {
+          uint32_t u[32];
+          tmem_ld32(tbase + q * P.n_mma + ch * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
+        }
         if (ch == nch - 1) {
           tc_fence_before();
           mbar_arrive(&c.tmem_empty[acc]);
@@ -297,7 +311,7 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
           }
         }
       }
-      if (++acc == 2) {
+      if (++acc == P.acc_bufs) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -345,6 +359,8 @@ void set_geometry(SplitKParams& P, int n_mma, int parts, int a_box_rows) {
   // inside the ring
   P.stage_bytes = std::max(P.a_bytes + P.parts_per_stage * P.b_bytes, BM * BK * 2);
   P.stages = std::min(kMaxStages, kRingBytes / P.stage_bytes);
+  P.acc_cols = P.parts_per_stage * n_mma;
+  P.acc_bufs = 2 * P.acc_cols <= static_cast<int>(TMEM_COLS) ? 2 : 1;
 }
 
 size_t smem_bytes(const SplitKParams& P) {
