@@ -215,17 +215,26 @@ def w4a16_bytes(cfg, ids):
 def launches_per_step(cfg):
     """Kernels one forward launches: router 3 (weight split, tensor-core
     logits, top-k), permute 2 (count/rank with the scan in its last block,
-    scatter), combine 1, plus the expert FFN path."""
+    scatter), combine 1, plus the expert FFN path and the shared expert's
+    launches when it does not ride in the routed ones."""
     n = 6
-    small_shared = cfg.I_s > 0 and cfg.T <= 32  # split-K GEMMs + slice sums for the shared expert
-    shared = (4 if small_shared else 2) if cfg.I_s > 0 else 0
-    if cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E:
-        n += 3 + shared          # routed: token prep + dequantising gate/up and down GEMMs
-    elif cfg.w4a16:
-        n += 4 + shared          # routed: (prep + gemv) x 2
-    else:
-        n += 2 + (4 if small_shared else 0)  # routed + large shared share two launches
-    return n
+    prefill = cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E   # int4 dequantised in shared memory, tensor cores
+    gemv = cfg.w4a16 and not prefill                      # int4 dequantised in registers
+    shared = 0
+    if cfg.I_s > 0:
+        if gemv and cfg.T <= 32:
+            shared = 0      # in the two GEMV launches
+        elif cfg.T <= 32:
+            shared = 4      # split-K GEMMs + ordered slice sums
+        elif cfg.w4a16:
+            shared = 2      # its own tcgen05 gate/up and down launches
+        else:
+            shared = 0      # one more problem of the routed tcgen05 launches
+    if prefill:
+        return n + 3 + shared  # token prep + dequantising gate/up and down
+    if gemv:
+        return n + 4 + shared  # (activation prep + GEMV) x 2
+    return n + 2 + shared      # gate/up + down
 
 
 def base_line(args, n_gpus, cfg):

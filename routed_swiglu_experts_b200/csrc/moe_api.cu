@@ -109,9 +109,12 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   const bool with_shared = x_shared != nullptr && Is > 0 && T > 0;
 
   // few tokens: the shared expert streams its weights with the split-K
-  // kernels; otherwise it is one more problem of the tcgen05 launches
-  const bool shared_small = with_shared && dense_small_ok(T, H, Is);
-  const bool shared_tc = with_shared && !shared_small;
+  // kernels -- or, beside the int4 GEMVs, inside their launches; otherwise it
+  // is one more problem of the tcgen05 launches
+  const bool gemv_path = is_int4(cfg) && !int4_prefill_preferred(R, E);
+  const bool shared_in_gemv = with_shared && gemv_path && w4a16_shared_fusable(T, Is);
+  const bool shared_small = with_shared && !shared_in_gemv && dense_small_ok(T, H, Is);
+  const bool shared_tc = with_shared && !shared_in_gemv && !shared_small;
   FfnProblem s_gu{}, s_d{};
   if (shared_tc) {
     s_gu = FfnProblem{x_shared, T, nullptr, 1, w.shared_w_gate_up, Is, H, hs, nullptr};
@@ -136,9 +139,11 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
       // gate/up in fp32 into the h region; the SwiGLU is applied while the
       // down projection's activations are prepared
       float* gu = at<float>(ws, L.h);
-      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, stream));
+      float* gu_s = shared_in_gemv ? at<float>(ws, L.small_part) : nullptr;
+      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, shared_in_gemv ? x_shared : nullptr, T,
+                                       gu_s, stream));
       if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
-      MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, stream));
+      MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, gu_s, T, hs, shared_out, stream));
     }
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, qd, sms, stream));
   }

@@ -86,10 +86,18 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
 
 // W4A16 routed expert kernels (dequantise in registers).
 // act16: scratch for the activations in MMA slot order (fp16, [rows, K]).
+// With x_shared != NULL (T <= kW4a16SharedMaxTokens tokens) the shared
+// expert's bf16 projections run in the same two launches: gate/up into
+// gu_shared (fp32 [T, 2 I_s]), its SwiGLU into h_shared (bf16 [T, I_s]) with
+// the down projection's activation prep, and down into shared_out.
+constexpr int kW4a16SharedMaxTokens = 32;
+bool w4a16_shared_fusable(int T, int Is);
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* gu, cudaStream_t stream);
+                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
+                                int T, float* gu_shared, cudaStream_t stream);
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
-                              int rows, void* act16, const float* w_perm, void* y_perm, cudaStream_t stream);
+                              int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
+                              int T, void* h_shared, void* shared_out, cudaStream_t stream);
 
 // W4A16 grouped GEMMs for many tokens per expert: int4 codes dequantised to
 // fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.

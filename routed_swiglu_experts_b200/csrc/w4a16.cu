@@ -105,10 +105,37 @@ __global__ void __launch_bounds__(256)
 // bf16 path's h, then laid out in MMA slot order as above.  gu: fp32
 // [rows, 2I] (gate columns [0, I), up columns [I, 2I)); one thread per 8
 // consecutive features of a row.
+// Shared expert (when gus != NULL): its fp32 gate/up [Ts, 2 I_s] from the
+// gate/up launch becomes h_s = bf16(silu(min(G, L)) * clamp(U, -L, L)) [Ts, I_s],
+// row-major, for the bf16 GEMV of its down projection (indices past n8).
+__device__ __forceinline__ float swiglu_clamped_f(float g, float u, float L) {
+  const float gc = fminf(g, L);
+  const float uc = fminf(fmaxf(u, -L), L);
+  return __fdividef(gc, 1.f + __expf(-gc)) * uc;
+}
+
 __global__ void __launch_bounds__(256)
-    w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16) {
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n8) return;
+    w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
+                             const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs) {
+  long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n8) {
+    idx -= n8;
+    if (gus == nullptr || idx >= n8s) return;
+    const int is8 = Is / 8;
+    const long long r = idx / is8;
+    const int f = static_cast<int>(idx - r * is8) * 8;
+    const float* gp = gus + r * 2 * Is + f;
+    float h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = swiglu_clamped_f(__ldg(gp + j), __ldg(gp + Is + j), L);
+    uint4 o;
+    o.x = pack_bf16x2(h[0], h[1]);
+    o.y = pack_bf16x2(h[2], h[3]);
+    o.z = pack_bf16x2(h[4], h[5]);
+    o.w = pack_bf16x2(h[6], h[7]);
+    *reinterpret_cast<uint4*>(hs + r * Is + f) = o;
+    return;
+  }
   const int i8 = I / 8;
   const long long r = idx / i8;
   const int f = static_cast<int>(idx - r * i8) * 8;
@@ -119,11 +146,7 @@ __global__ void __launch_bounds__(256)
   const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
   float h[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float gc = fminf(gv[j], L);
-    const float uc = fminf(fmaxf(uv[j], -L), L);
-    h[j] = __bfloat162float(__float2bfloat16_rn(__fdividef(gc, 1.f + __expf(-gc)) * uc));
-  }
+  for (int j = 0; j < 8; ++j) h[j] = __bfloat162float(__float2bfloat16_rn(swiglu_clamped_f(gv[j], uv[j], L)));
   const __half2 a04 = __floats2half2_rn(h[0], h[4]);
   const __half2 b15 = __floats2half2_rn(h[1] * 0.0625f, h[5] * 0.0625f);
   const __half2 a26 = __floats2half2_rn(h[2], h[6]);
@@ -135,6 +158,85 @@ __global__ void __launch_bounds__(256)
   o.w = *reinterpret_cast<const uint32_t*>(&b37);
   act16[idx] = o;
 }
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The shared expert's bf16 projection for up to 32 tokens, run by the
+// blocks of blockIdx.y == 0 of the routed GEMV launches so that its weight
+// stream (HBM-bound, no dequantisation) overlaps the routed experts' ALU-bound
+// one instead of running before them.  One warp: rows [n0, n0 + 16) of
+// W [N, K] against every token of act [T, K] (bf16, row-major), fp32
+// accumulation, out [T, N] (fp32, or bf16 when !F32OUT).
+// Each thread loads 8 consecutive k of its rows g and g + 8 and of its tokens
+// per 32-wide K step and feeds two m16n8k16 MMAs per 8 tokens; the MMA reduces
+// over its 16 slots, so physical k = k0 + 8t + j goes to slot 2t + {0, 1, 8, 9}
+// (j = 0..3) of the first MMA and the same slots of the second (j = 4..7),
+// for weights and activations alike.
+template <bool F32OUT>
+__device__ __noinline__ void shared_gemv_warp(const __nv_bfloat16* __restrict__ W, const __nv_bfloat16* __restrict__ act,
+                                              int N, int K, int T, int n0, void* __restrict__ out, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  float acc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const bool r0 = n0 + g < N, r8 = n0 + g + 8 < N;
+  const uint4* w0 = reinterpret_cast<const uint4*>(W + static_cast<size_t>(r0 ? n0 + g : 0) * K + 8 * t);
+  const uint4* w8 = reinterpret_cast<const uint4*>(W + static_cast<size_t>(r8 ? n0 + g + 8 : 0) * K + 8 * t);
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  // the weight rows of the next K step are loaded before this step's MMAs
+  // (two steps of weights in flight per thread)
+  auto load_w = [&](int k0, uint4& a, uint4& b) {
+    const bool kin = k0 < K && k0 + 8 * t < K;  // K % 8 == 0: the 8 values are all in or all out
+    a = (r0 && kin) ? __ldcs(w0 + k0 / 8) : z;
+    b = (r8 && kin) ? __ldcs(w8 + k0 / 8) : z;
+  };
+  uint4 na, nb;
+  load_w(0, na, nb);
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    const bool kin = k0 + 8 * t < K;
+    const uint4 wa = na, wb = nb;
+    load_w(k0 + 32, na, nb);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tok = 8 * j + g;
+      const uint4 av = (tok < T && kin)
+                           ? __ldg(reinterpret_cast<const uint4*>(act + static_cast<size_t>(tok) * K + k0 + 8 * t))
+                           : z;
+      mma_bf16_16816(acc[j], wa.x, wb.x, wa.y, wb.y, av.x, av.y);
+      mma_bf16_16816(acc[j], wa.z, wb.z, wa.w, wb.w, av.z, av.w);
+    }
+  }
+  // acc[j][0..1]: row n0 + g, tokens 8j + 2t + {0, 1}; acc[j][2..3]: row n0 + g + 8
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int tok = 8 * j + 2 * t + (c & 1);
+      const int col = n0 + g + 8 * (c >> 1);
+      if (tok < T && col < N) {
+        const size_t o = static_cast<size_t>(tok) * N + col;
+        if (F32OUT)
+          static_cast<float*>(out)[o] = acc[j][c];
+        else
+          static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(acc[j][c]);
+      }
+    }
+}
+
+// Shared-expert projection riding along in a routed GEMV launch (NULL w: none).
+struct SharedJob {
+  const __nv_bfloat16* w;    // [N, K]
+  const __nv_bfloat16* act;  // [T, K]
+  void* out;                 // [T, N]: fp32 (gate/up) or bf16 (down)
+  int N, K, T;
+};
 
 // Streaming GEMV.  One warp owns 16 output rows of one expert for one
 // 8-token chunk and walks K one 128-wide scale group at a time.  The code
@@ -165,10 +267,20 @@ template <bool F32OUT>
 __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
     w4a16_gemv_kernel(const uint4* __restrict__ act16, const int32_t* __restrict__ offsets,
                       const uint8_t* __restrict__ q, const __nv_bfloat16* __restrict__ scales, int N, int K,
-                      const float* __restrict__ w_perm, void* __restrict__ out) {
+                      const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj) {
   extern __shared__ uint4 gemv_ring[];
   constexpr int S = kGemvStages;
-  const int e = blockIdx.y;
+  // blocks of the first grid row take the shared expert (when there is one):
+  // they start first, and their weight stream runs beside the routed blocks'
+  int e = blockIdx.y;
+  if (sj.w != nullptr) {
+    if (e == 0) {
+      const int n0s = blockIdx.x * kGemvRows + (threadIdx.x / 32) * 16;
+      if (n0s < sj.N) shared_gemv_warp<F32OUT>(sj.w, sj.act, sj.N, sj.K, sj.T, n0s, sj.out, threadIdx.x % 32);
+      return;
+    }
+    --e;
+  }
   const int r_begin = offsets[e], r_end = offsets[e + 1];
   if (r_end <= r_begin) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -280,36 +392,52 @@ cudaError_t launch_prep(const void* act, int rows, int K, void* act16, cudaStrea
 
 template <bool F32OUT>
 cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, const void* act16,
-                        const int32_t* offsets, const float* w_perm, void* out, cudaStream_t stream) {
-  const dim3 grid((N + kGemvRows - 1) / kGemvRows, E);
+                        const int32_t* offsets, const float* w_perm, void* out, const SharedJob& sj,
+                        cudaStream_t stream) {
+  const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
+  const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
   w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, kGemvSmem, stream>>>(
       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
-      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out);
+      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+bool w4a16_shared_fusable(int T, int Is) { return Is > 0 && T >= 1 && T <= kW4a16SharedMaxTokens; }
+
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* gu, cudaStream_t stream) {
+                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
+                                int T, float* gu_shared, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
   cudaError_t e = launch_prep(x_perm, rows, H, act16, stream);
   if (e != cudaSuccess) return e;
+  SharedJob sj{};
+  if (x_shared != nullptr)  // shared gate/up [2 I_s, H] x tokens [T, H] -> fp32 [T, 2 I_s]
+    sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_gate_up), static_cast<const __nv_bfloat16*>(x_shared),
+                   gu_shared, 2 * cfg.shared_inter, H, T};
   // W_gu [E, 2I, H/2]: one matrix of 2I rows per expert (gate rows, then up rows)
-  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, stream);
+  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, sj, stream);
 }
 
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
-                              int rows, void* act16, const float* w_perm, void* y_perm, cudaStream_t stream) {
-  const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
+                              int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
+                              int T, void* h_shared, void* shared_out, cudaStream_t stream) {
+  const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts, Is = cfg.shared_inter;
   const long long n8 = static_cast<long long>(rows) * (I / 8);
-  if (n8 > 0) {
-    w4a16_prep_swiglu_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-        gu, I, n8, cfg.swiglu_limit, static_cast<uint4*>(act16));
+  const long long n8s = gu_shared != nullptr ? static_cast<long long>(T) * (Is / 8) : 0;
+  if (n8 + n8s > 0) {
+    w4a16_prep_swiglu_kernel<<<static_cast<unsigned>((n8 + n8s + 255) / 256), 256, 0, stream>>>(
+        gu, I, n8, cfg.swiglu_limit, static_cast<uint4*>(act16), gu_shared, Is, n8s,
+        static_cast<__nv_bfloat16*>(h_shared));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, stream);
+  SharedJob sj{};
+  if (gu_shared != nullptr)  // shared down [H, I_s] x h_s [T, I_s] -> bf16 [T, H], unscaled
+    sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_down), static_cast<const __nv_bfloat16*>(h_shared),
+                   shared_out, H, Is, T};
+  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, sj, stream);
 }
 
 }  // namespace moe

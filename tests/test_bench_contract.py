@@ -30,9 +30,8 @@ def test_gemm_flops_of_the_mid_layer():
     # gate/up + down (shared expert as a second problem), combine
     ("mid", 8),
     ("large_prefill", 8),
-    # ... + shared expert by split-K (2 GEMMs + 2 slice sums) + W4A16 (prep +
-    # GEMV) x 2
-    ("decode_w4a16", 14),
+    # ... + W4A16 (prep + GEMV) x 2, the shared expert inside the GEMV launches
+    ("decode_w4a16", 10),
     # ... + token prep + dequantising gate/up and down + bf16 shared gate/up
     # and down launches
     ("prefill_w4a16", 11),
