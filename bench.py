@@ -48,6 +48,10 @@ def parse_args(argv=None):
     ap.add_argument("--graph", action="store_true", help="replay the forward from a captured CUDA graph")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the W4A16 decode-layer measurement added beside the mid layer's line")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: every rank runs the whole layer on its own tokens (weak scaling); "
+                         "ep: expert parallelism, every rank holds E/N experts and 1/N of the shared expert for "
+                         "the same tokens, one all-reduce per step (strong scaling)")
     return ap.parse_args(argv)
 
 
@@ -556,6 +560,102 @@ def bench_ours(args, rank, world, local_rank):
     return line
 
 
+# ------------------------------------------------ expert parallel arm ----
+
+def bench_ep(args, rank, world, local_rank):
+    """Expert parallelism: every rank holds the full router, its contiguous
+    range of E/N experts and 1/N of the shared expert's intermediate
+    features, runs moe_forward_ep on all T tokens and joins the ranks'
+    partial sums with one NCCL all-reduce (page "Module glm5next_mlp",
+    §One all-reduce for both EP and TP).  Total work per step is fixed
+    (strong scaling): value = T / step time."""
+    import torch
+    import torch.distributed as dist
+    import routed_swiglu_experts_b200 as rse
+    from routed_swiglu_experts_b200 import ep
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    rse.load_library()
+    cfg, inp = make_inputs(args.workload)
+    c = cfg
+
+    def mv(t):
+        return None if t is None else t.to(dev)
+    group = dist.group.WORLD if world > 1 else None
+    layer = ep.ExpertParallelLayer(
+        hidden=c.H, num_experts=c.E, top_k=c.k, expert_inter=c.I, shared_inter=c.I_s,
+        swiglu_limit=c.swiglu_limit, routed_scaling_factor=c.alpha, renormalize=c.renorm,
+        router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias), w_gate_up=mv(inp.w_gate_up),
+        w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up), s_down=mv(inp.s_down),
+        shared_w_gate_up=mv(inp.shared_w_gate_up), shared_w_down=mv(inp.shared_w_down),
+        rank=rank, world=world, max_tokens=c.T, group=group)
+    x = inp.x.to(dev)
+    out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(gpu_uuid(dev))
+    for _ in range(args.warmup):
+        layer.forward(x, out=out)
+    torch.cuda.synchronize()
+    rank_barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    rank_barrier(world)
+    ms_per_step = rank_max(e0.elapsed_time(e1), world, dev) / args.steps
+
+    # end to end: the step's tokens from pinned host memory, its result back
+    x_host = inp.x.pin_memory()
+    out_host = torch.empty(c.T, c.H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    rank_barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    rank_barrier(world)
+    e2e_ms = rank_max(e0.elapsed_time(e1), world, dev) / args.steps
+    clk = clocks.finish()
+    assert layer.device_error() == 0
+    b, e = layer.expert_range
+    line = base_line(args, world, c)
+    line["scaling"] = "strong"
+    line["config"]["tokens_per_gpu_step"] = c.T
+    line["config"]["global_tokens_per_step"] = c.T
+    line["config"]["parallelism"] = (f"ep{world}: experts split in contiguous ranges (rank 0: [{b}, {e})), shared "
+                                     f"expert split by intermediate features, router replicated, one NCCL "
+                                     f"all-reduce of the bf16 [T, H] partials per step")
+    line.update({
+        "mode": "ep", "value": c.T / (ms_per_step / 1e3), "ms_per_step": ms_per_step, "dtype": "bf16",
+        "e2e": {"value": c.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "method": "per step: input copied from pinned host memory, moe_forward_ep + all-reduce, result "
+                          "copied back, one stream",
+                "h2d_bytes_per_step": c.T * c.H * 2, "d2h_bytes_per_step": c.T * c.H * 2},
+        "gpu_launches": launches_per_step(c) * args.steps,
+        "clocks": clk,
+        "roofline": None,
+        "note": "the roofline object is reported by the replicas mode (one GPU runs the whole layer)",
+    })
+    return line
+
+
 # -------------------------------------------------------- reference arm ----
 
 def bench_reference(args):
@@ -607,7 +707,8 @@ def main(argv=None):
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        line = bench_ours(args, rank, world, local_rank)
+        line = bench_ep(args, rank, world, local_rank) if args.mode == "ep" else bench_ours(args, rank, world,
+                                                                                           local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

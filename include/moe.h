@@ -225,6 +225,39 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
                        int32_t* topk_ids_opt, float* topk_w_opt,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Expert-parallel forward of one rank ([glm5next] §One all-reduce for both EP
+ * and TP: each rank combines the shared output and its local routed slots,
+ * then one all-reduce of the [T, H] partial sums gives the layer output;
+ * the router is replicated and ranks all experts, and the ranks' expert
+ * ranges partition [0, E)).
+ *   out_partial[t] = bf16( shared_r(x[t])
+ *                          + sum over slots j with expert_begin <= e_j < expert_end
+ *                            of w_j * FFN_{e_j}(x[t]) )
+ * summed in fp32 in slot order, where shared_r is this rank's slice of the
+ * shared expert (its SwiGLU is per intermediate feature, so a slice of the
+ * intermediate dimension is a narrower shared expert, and the slices' down
+ * projections add up to the whole).  Adding the ranks' out_partial gives
+ * moe_forward's output (up to rounding) when their expert ranges partition
+ * [0, E) and their shared slices partition [0, I_s).
+ *   cfg   as for moe_forward, except cfg->shared_inter = this rank's slice
+ *         width of the shared intermediate (0: no shared work on this rank);
+ *         cfg->num_experts is the full E (the router ranks every expert).
+ *   w     router_w / correction_bias: the full [E, H] / [E];
+ *         w_gate_up, w_down (and s_gate_up, s_down): the LOCAL experts only,
+ *         [expert_end - expert_begin, ...], local expert 0 = global expert
+ *         expert_begin (may be NULL when the range is empty);
+ *         shared_w_gate_up [2 I_s_local, H] (the slice's gate rows, then its
+ *         up rows) and shared_w_down [H, I_s_local] (the slice's columns).
+ *   0 <= expert_begin <= expert_end <= E, else MOE_ERR_INVALID_ARG.
+ *   x bf16 [T, H] (every rank gets all T tokens); out_partial bf16 [T, H].
+ *   topk_ids_opt / topk_w_opt: as for moe_forward (every token's selection).
+ * The workspace is sized by moe_workspace_size(cfg, T) with this rank's cfg.
+ * The all-reduce itself is the caller's (NCCL over NVLink, one call). */
+MOE_API moe_status moe_forward_ep(const moe_config* cfg, const moe_weights* w, int32_t expert_begin,
+                                  int32_t expert_end, const void* x, int32_t T, void* out_partial,
+                                  int32_t* topk_ids_opt, float* topk_w_opt, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
 /* Permute without a workspace, for callers that may not allocate device
  * memory on their enqueue path (framework / inference-server plugins and
  * serving loops that own all device memory and only pass their own input

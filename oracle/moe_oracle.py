@@ -272,3 +272,34 @@ def moe_forward(layer, tokens: Optional[Sequence[int]] = None,
         out += sel.weights[:, j:j + 1] * y_perm[rows[:, j]]
     return LayerResult(out, sel, perm, y_perm, h_perm, shared,
                        shared_h if keep_hidden else None, tok)
+
+
+# ------------------------------------------------- expert parallelism ----
+
+def moe_partial(layer, expert_begin: int, expert_end: int, shared_begin: int, shared_end: int,
+                tokens: Optional[Sequence[int]] = None,
+                ids_override: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One rank's partial sum under expert parallelism ([glm5next] §One
+    all-reduce for both EP and TP: each rank adds the shared output and its
+    local routed slots in its combine; one all-reduce of the [T, H] partials
+    gives the layer output).  The rank owns routed experts
+    [expert_begin, expert_end) and the shared expert's intermediate features
+    [shared_begin, shared_end): the clamped SwiGLU acts feature by feature, so
+    the shared output is the sum over feature slices of W_down[:, slice]
+    h[slice].  The router is the full one (every rank ranks all experts).
+      out_r[t] = sum_{f in slice} W_sd[:, f] h_s[t, f]
+                 + sum_{j : expert_begin <= e_j < expert_end} w[t, j] FFN_{e_j}(x[t])
+    fp64 [T, H]."""
+    res = moe_forward(layer, tokens=tokens, keep_hidden=True, ids_override=ids_override)
+    T = res.out.shape[0]
+    H, k = layer.cfg.H, layer.cfg.k
+    out = torch.zeros(T, H, dtype=f64)
+    if layer.cfg.I_s > 0 and shared_end > shared_begin:
+        sd = _cpu64(layer.shared_w_down)
+        out += res.shared_h[:, shared_begin:shared_end] @ sd[:, shared_begin:shared_end].T
+    rows = res.perm.row_of.view(T, k)
+    ids = res.selection.ids
+    for j in range(k):
+        local = ((ids[:, j] >= expert_begin) & (ids[:, j] < expert_end)).to(f64)[:, None]
+        out += local * res.selection.weights[:, j:j + 1] * res.y_perm[rows[:, j]]
+    return out

@@ -31,7 +31,7 @@ MOE_INT4_MAX_SWIGLU_LIMIT = 255.0
 
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",
-    "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward",
+    "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_forward_ep",
     "moe_read_device_error", "moe_permute_no_alloc", "moe_selftest_device_timeout", "moe_selftest_pair_timeout",
 )
 MOE_NO_ALLOC_MAX_ROWS = 131072
@@ -98,6 +98,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_swiglu_ffn": (ctypes.c_int, [CFG, W, P, P, P, I32, P, P, P, P, SZ, P]),
         "moe_combine": (ctypes.c_int, [CFG, P, P, P, P, I32, P, P]),
         "moe_forward": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, SZ, P]),
+        "moe_forward_ep": (ctypes.c_int, [CFG, W, I32, I32, P, I32, P, P, P, P, SZ, P]),
         "moe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(I32)]),
         "moe_selftest_device_timeout": (ctypes.c_int, [P, SZ, P]),
         "moe_selftest_pair_timeout": (ctypes.c_int, [P, SZ, I32, P]),
@@ -201,6 +202,12 @@ def moe_forward(cfg, w, x, T, out, topk_ids_opt, topk_w_opt, ws, stream=None):
     _check(load_library().moe_forward(ctypes.byref(cfg), ctypes.byref(w), _ptr(x), int(T), _ptr(out),
                                       _ptr(topk_ids_opt), _ptr(topk_w_opt), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def moe_forward_ep(cfg, w, expert_begin, expert_end, x, T, out_partial, topk_ids_opt, topk_w_opt, ws, stream=None):
+    _check(load_library().moe_forward_ep(ctypes.byref(cfg), ctypes.byref(w), int(expert_begin), int(expert_end),
+                                         _ptr(x), int(T), _ptr(out_partial), _ptr(topk_ids_opt), _ptr(topk_w_opt),
+                                         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_forward_ep")
 
 
 def moe_permute_no_alloc(cfg, topk_ids, topk_w, x, T, expert_offsets, row_of, src, w_perm, x_perm, stream=None):

@@ -1,7 +1,8 @@
 // Combine ("Module glm5next_mlp", §One all-reduce for both EP and TP: the
 // shared output and the routed slots are added in one combine kernel):
 //   out[t] = bf16( shared[t] + sum_j c_j * y_perm[row_of[t*k + j]] ),
-// fp32 sum in slot order.  One warp per token, 16-byte vectors.
+// fp32 sum in slot order (the shared row first).  One warp per token,
+// 16-byte vectors.
 #include "moe_internal.h"
 
 namespace moe {
@@ -19,25 +20,38 @@ __device__ __forceinline__ void add8(float (&a)[8], const uint4 v, float c) {
   a[7] = fmaf(c, bf16hi(v.w), a[7]);
 }
 
-// One warp per (token, 256-element chunk of the hidden row): 8 warps per
-// block, so even a handful of tokens spreads over many SMs.
-__global__ void __launch_bounds__(256)
+// One warp per token: lane j < k reads slot j's routed row and weight once,
+// the warp shares them with shuffles, then walks the hidden row two 16-byte
+// vectors per lane at a time, so every lane keeps (k + 1) x 2 loads in flight
+// and the index work is paid once per token.  Routed rows outside [lo, hi)
+// (when `range` is given: range[0] = lo, range[e1 - e0] = hi, the rows of this
+// rank's experts) are left out: expert parallelism's partial combine.
+constexpr int kCombineWarps = 8;
+constexpr int kVecPerLane = 2;
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ row_of,
                    const float* __restrict__ topk_w, const __nv_bfloat16* __restrict__ shared, int T, int k, int H,
-                   int blocks_per_token, __nv_bfloat16* __restrict__ out) {
+                   const int32_t* __restrict__ range, int range_len, __nv_bfloat16* __restrict__ out) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x / blocks_per_token;
-  const int chunk = (blockIdx.x - t * blocks_per_token) * 8 + warp;
+  const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= T) return;
-  const int c = chunk * 32 + lane;  // 16-byte column of the row
-  if (chunk * 32 >= H / 8) return;  // whole warp past the row
-  // slot rows and weights: one load per lane, then broadcast to every lane
+  int lo = 0, hi = 0x7fffffff;
+  if (range != nullptr) {
+    lo = __ldg(range);
+    hi = __ldg(range + range_len);
+  }
+  // slot rows and weights: one load per lane, then broadcast to every lane;
+  // `used` marks the slots whose row is in [lo, hi)
   int my_row = 0;
   float my_c = 1.f;
+  bool mine = false;
   if (lane < k) {
-    my_row = row_of[static_cast<size_t>(t) * k + lane];
-    if (topk_w != nullptr) my_c = topk_w[static_cast<size_t>(t) * k + lane];
+    my_row = __ldg(row_of + static_cast<size_t>(t) * k + lane);
+    mine = my_row >= lo && my_row < hi;
+    if (topk_w != nullptr) my_c = __ldg(topk_w + static_cast<size_t>(t) * k + lane);
   }
+  const uint32_t used = __ballot_sync(0xffffffffu, mine);
   int rows[MOE_MAX_TOP_K];
   float cs[MOE_MAX_TOP_K];
 #pragma unroll
@@ -45,29 +59,56 @@ __global__ void __launch_bounds__(256)
     rows[j] = __shfl_sync(0xffffffffu, my_row, j);
     cs[j] = __shfl_sync(0xffffffffu, my_c, j);
   }
-  if (c >= H / 8) return;
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (shared != nullptr) add8(a, __ldg(reinterpret_cast<const uint4*>(shared + static_cast<size_t>(t) * H) + c), 1.f);
+  const int n16 = H / 8;  // 16-byte vectors per row
+  const uint4* srow = shared != nullptr ? reinterpret_cast<const uint4*>(shared + static_cast<size_t>(t) * H) : nullptr;
+  uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H);
+  for (int c0 = lane; c0 < n16; c0 += 32 * kVecPerLane) {
+    float a[kVecPerLane][8];
 #pragma unroll
-  for (int j = 0; j < MOE_MAX_TOP_K; ++j)
-    if (j < k) add8(a, __ldg(reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(rows[j]) * H) + c), cs[j]);
-  uint4 o;
-  o.x = pack_bf16x2(a[0], a[1]);
-  o.y = pack_bf16x2(a[2], a[3]);
-  o.z = pack_bf16x2(a[4], a[5]);
-  o.w = pack_bf16x2(a[6], a[7]);
-  reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = o;
+    for (int v = 0; v < kVecPerLane; ++v)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) a[v][q] = 0.f;
+    if (srow != nullptr) {
+#pragma unroll
+      for (int v = 0; v < kVecPerLane; ++v) {
+        const int c = c0 + 32 * v;
+        if (c < n16) add8(a[v], __ldg(srow + c), 1.f);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOP_K; ++j) {
+      if ((used >> j) & 1u) {
+        const uint4* yr = reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(rows[j]) * H);
+#pragma unroll
+        for (int v = 0; v < kVecPerLane; ++v) {
+          const int c = c0 + 32 * v;
+          if (c < n16) add8(a[v], __ldg(yr + c), cs[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < kVecPerLane; ++v) {
+      const int c = c0 + 32 * v;
+      if (c < n16) {
+        uint4 o;
+        o.x = pack_bf16x2(a[v][0], a[v][1]);
+        o.y = pack_bf16x2(a[v][2], a[v][3]);
+        o.z = pack_bf16x2(a[v][4], a[v][5]);
+        o.w = pack_bf16x2(a[v][6], a[v][7]);
+        orow[c] = o;
+      }
+    }
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
-                           const void* shared_out, int T, void* out, cudaStream_t stream) {
-  const int chunks = (cfg.hidden / 8 + 31) / 32;  // 256-element chunks per row
-  const int bpt = (chunks + 7) / 8;
-  combine_kernel<<<static_cast<unsigned>(T) * bpt, 256, 0, stream>>>(
+                           const void* shared_out, int T, void* out, const int32_t* range, int range_len,
+                           cudaStream_t stream) {
+  combine_kernel<<<static_cast<unsigned>((T + kCombineWarps - 1) / kCombineWarps), kCombineWarps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(y_perm), row_of, topk_w, static_cast<const __nv_bfloat16*>(shared_out), T,
-      cfg.top_k, cfg.hidden, bpt, static_cast<__nv_bfloat16*>(out));
+      cfg.top_k, cfg.hidden, range, range_len, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 

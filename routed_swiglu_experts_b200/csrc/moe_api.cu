@@ -94,12 +94,17 @@ moe_status check_router_weights(const moe_weights* w) {
   } while (0)
 
 // The grouped FFN on already-permuted rows (routed) plus, optionally, the
-// shared expert on the raw tokens.
+// shared expert on the raw tokens.  cfg.num_experts is the number of experts
+// this call computes (0 allowed: shared expert only), `offsets` their
+// [E + 1] row offsets (absolute rows of x_perm), and w's routed weights hold
+// exactly those experts; e_total is the router's expert count (the int4 path
+// picks its kernel by the average routed rows per expert, R / e_total).
 moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_perm, const int32_t* offsets,
                    const float* w_perm, int32_t T, void* y_perm, const void* x_shared, void* shared_out, void* ws,
-                   const WsLayout& L, cudaStream_t stream) {
+                   const WsLayout& L, cudaStream_t stream, int e_total) {
   const int H = cfg.hidden, I = cfg.expert_inter, Is = cfg.shared_inter, E = cfg.num_experts;
   const int R = T * cfg.top_k;
+  const bool routed = E > 0;
   int32_t* err = err_word(ws);
   int32_t* qgu = tile_queue(ws, kQueueGateUp);
   int32_t* qd = tile_queue(ws, kQueueDown);
@@ -111,7 +116,8 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   // few tokens: the shared expert streams its weights with the split-K
   // kernels -- or, beside the int4 GEMVs, inside their launches; otherwise it
   // is one more problem of the tcgen05 launches
-  const bool gemv_path = is_int4(cfg) && !int4_prefill_preferred(R, E);
+  const bool prefill_path = is_int4(cfg) && int4_prefill_preferred(R, e_total);
+  const bool gemv_path = is_int4(cfg) && !prefill_path;
   const bool shared_in_gemv = with_shared && gemv_path && w4a16_shared_fusable(T, Is);
   const bool shared_small = with_shared && !shared_in_gemv && dense_small_ok(T, H, Is);
   const bool shared_tc = with_shared && !shared_in_gemv && !shared_small;
@@ -126,14 +132,16 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
   if (!is_int4(cfg)) {
     FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
-    MOE_CUDA_TRY(launch_gemm_gateup(&r_gu, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, qgu, sms, stream));
-    MOE_CUDA_TRY(launch_gemm_down(&r_d, shared_tc ? &s_d : nullptr, err, qd, sms, stream));
+    MOE_CUDA_TRY(launch_gemm_gateup(routed ? &r_gu : nullptr, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, qgu,
+                                    sms, stream));
+    MOE_CUDA_TRY(launch_gemm_down(routed ? &r_d : nullptr, shared_tc ? &s_d : nullptr, err, qd, sms, stream));
   } else {
     void* act16 = at<void>(ws, L.act16);
-    if (int4_prefill_preferred(R, E)) {
+    if (prefill_path) {
       // many tokens per expert: dequantise in shared memory, tensor cores
-      MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_perm, offsets, R, act16, at<void>(ws, L.h), w_perm, y_perm,
-                                           err, tile_queue(ws, kQueueInt4GateUp), sms, stream));
+      if (routed)
+        MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_perm, offsets, R, act16, at<void>(ws, L.h), w_perm, y_perm,
+                                             err, tile_queue(ws, kQueueInt4GateUp), sms, stream));
       if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
     } else {
       // gate/up in fp32 into the h region; the SwiGLU is applied while the
@@ -310,7 +318,8 @@ moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weights* w, c
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
-  return run_ffn(*cfg, *w, x_perm, expert_offsets, w_perm, T, y_perm, x_shared, shared_out, ws, L, stream);
+  return run_ffn(*cfg, *w, x_perm, expert_offsets, w_perm, T, y_perm, x_shared, shared_out, ws, L, stream,
+                 cfg->num_experts);
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
@@ -322,7 +331,7 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
   if (topk_w != nullptr && !aligned16(topk_w)) return MOE_ERR_INVALID_ARG;
   if (shared_out != nullptr && !aligned16(shared_out)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  return from_cuda(launch_combine(*cfg, y_perm, row_of, topk_w, shared_out, T, out, stream));
+  return from_cuda(launch_combine(*cfg, y_perm, row_of, topk_w, shared_out, T, out, nullptr, 0, stream));
 }
 
 moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* x, int32_t T, void* out,
@@ -352,8 +361,48 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   void* y_perm = at<void>(ws, L.y_perm);
   const bool shared = cfg->shared_inter > 0;
   void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;
-  MOE_TRY(run_ffn(*cfg, *w, x_perm, offsets, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws, L, stream));
-  return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out, stream));
+  MOE_TRY(run_ffn(*cfg, *w, x_perm, offsets, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws, L, stream,
+                  cfg->num_experts));
+  return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out, nullptr, 0, stream));
+}
+
+moe_status moe_forward_ep(const moe_config* cfg, const moe_weights* w, int32_t expert_begin, int32_t expert_end,
+                          const void* x, int32_t T, void* out_partial, int32_t* topk_ids_opt, float* topk_w_opt,
+                          void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_router_weights(w));
+  if (expert_begin < 0 || expert_end < expert_begin || expert_end > cfg->num_experts) return MOE_ERR_INVALID_ARG;
+  const int El = expert_end - expert_begin;
+  if (El > 0) MOE_TRY(check_expert_weights(*cfg, w));
+  MOE_TRY(check_shared_weights(*cfg, w));
+  if (x == nullptr || out_partial == nullptr || !aligned16(x) || !aligned16(out_partial)) return MOE_ERR_INVALID_ARG;
+  if ((topk_ids_opt != nullptr && !aligned16(topk_ids_opt)) || (topk_w_opt != nullptr && !aligned16(topk_w_opt)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  int32_t* ids = topk_ids_opt != nullptr ? topk_ids_opt : at<int32_t>(ws, L.ids);
+  float* wts = topk_w_opt != nullptr ? topk_w_opt : at<float>(ws, L.wts);
+  // the router ranks every expert ([glm5next]: it is given the full count)
+  MOE_CUDA_TRY(launch_router(*cfg, *w, x, T, ids, wts, at<float>(ws, L.logits), at<void>(ws, L.w_split),
+                             err_word(ws), num_sms_current_device(), stream));
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  float* w_perm = at<float>(ws, L.w_perm);
+  void* x_perm = at<void>(ws, L.x_perm);
+  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, at<int32_t>(ws, L.src), w_perm, x_perm,
+                              at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), perm_ticket(ws), stream,
+                              expert_begin, expert_end));
+  void* y_perm = at<void>(ws, L.y_perm);
+  const bool shared = cfg->shared_inter > 0;
+  void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;
+  moe_config local = *cfg;
+  local.num_experts = El;
+  MOE_TRY(run_ffn(local, *w, x_perm, offsets + expert_begin, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws,
+                  L, stream, cfg->num_experts));
+  return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out_partial, offsets + expert_begin,
+                                  El, stream));
 }
 
 moe_status moe_selftest_device_timeout(void* scratch, size_t scratch_bytes, moe_stream_t stream) {

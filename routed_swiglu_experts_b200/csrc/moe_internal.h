@@ -57,12 +57,18 @@ constexpr int kPermChunk = 2048;
 inline int perm_blocks(int R) { return std::max(1, (R + kPermChunk - 1) / kPermChunk); }
 // block_base: [perm_blocks(T*k) * E] scratch; local_rank: [T*k] scratch;
 // done: a ticket counter that is zero before the launch and left at zero.
+// Hidden rows are copied into x_perm only for experts in [e0, e1) (e1 < 0:
+// every expert); the maps and weights cover every slot.
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
                            int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
-                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream);
+                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream, int e0 = 0,
+                           int e1 = -1);
 
+// range: NULL, or device pointer to expert offsets: only routed rows in
+// [range[0], range[range_len]) are added (expert parallelism's partial combine).
 cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
-                           const void* shared_out, int T, void* out, cudaStream_t stream);
+                           const void* shared_out, int T, void* out, const int32_t* range, int range_len,
+                           cudaStream_t stream);
 
 // Grouped GEMMs (tcgen05).  One "problem" is a set of row groups that share
 // an A operand tensor and a weight tensor; the routed experts are one problem

@@ -159,13 +159,14 @@ __global__ void __launch_bounds__(kPermWarps * 32)
   if (threadIdx.x == 0) *done = 0;  // ready for the next launch
 }
 
-// One warp per slot: routed row, inverse maps, weight, and the hidden row.
+// One warp per slot: routed row, inverse maps, weight, and the hidden row
+// (copied only for experts in [e0, e1): the experts this call computes).
 __global__ void __launch_bounds__(256)
     perm_scatter_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w,
                         const __nv_bfloat16* __restrict__ x, int R, int k, int E, int H,
                         const int32_t* __restrict__ block_base, const int32_t* __restrict__ local_rank,
                         int32_t* __restrict__ row_of, int32_t* __restrict__ src, float* __restrict__ w_perm,
-                        __nv_bfloat16* __restrict__ x_perm) {
+                        __nv_bfloat16* __restrict__ x_perm, int e0, int e1) {
   const int i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (i >= R) return;
@@ -176,6 +177,7 @@ __global__ void __launch_bounds__(256)
     src[row] = i;
     w_perm[row] = topk_w[i];
   }
+  if (id < e0 || id >= e1) return;
   const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<size_t>(i / k) * H);
   uint4* d = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * H);
   const int n16 = H / 8;
@@ -194,7 +196,8 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
                            int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
-                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream) {
+                           int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream, int e0,
+                           int e1) {
   const int E = cfg.num_experts, k = cfg.top_k, H = cfg.hidden;
   const int R = T * k;
   const int nb = perm_blocks(R);
@@ -207,7 +210,8 @@ cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const floa
   perm_count_rank_kernel<<<nb, kPermWarps * 32, smem, stream>>>(ids, R, E, block_base, local_rank, offsets, done);
   perm_scatter_kernel<<<(R + 7) / 8, 256, 0, stream>>>(ids, topk_w, static_cast<const __nv_bfloat16*>(x), R, k, E,
                                                        H, block_base, local_rank, row_of, src, w_perm,
-                                                       static_cast<__nv_bfloat16*>(x_perm));
+                                                       static_cast<__nv_bfloat16*>(x_perm), e0,
+                                                       e1 < 0 ? E : e1);
   return cudaGetLastError();
 }
 

@@ -396,6 +396,7 @@ cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, 
                         cudaStream_t stream) {
   const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
   const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
+  if (grid.y == 0) return cudaSuccess;  // no routed expert and no shared expert in this call
   w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, kGemvSmem, stream>>>(
       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
       static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);

@@ -197,3 +197,26 @@ def test_pair_selftest_argument_checks(lib):
     assert lib.moe_selftest_pair_timeout(FAKE + 16, n, _abi.MOE_SELFTEST_PAIR_INT4, None) == _abi.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_pair_timeout(FAKE, n, 2, None) == _abi.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_pair_timeout(FAKE, n, -1, None) == _abi.MOE_ERR_INVALID_ARG
+
+
+def _call_ep(lib, cfg, w, b, e, T=16, x=FAKE, out=FAKE, ws=FAKE):
+    ok = _abi.moe_config_validate(cfg) == _abi.MOE_OK
+    nbytes = _abi.moe_workspace_size(cfg, max(T, 0)) if ok else 1 << 40
+    return lib.moe_forward_ep(ctypes.byref(cfg), ctypes.byref(w), b, e, x, T, out, None, None, ws, nbytes, None)
+
+
+def test_forward_ep_argument_checks(lib):
+    """The expert range must lie in [0, E]; an empty range needs no routed
+    weights; everything is validated before any launch."""
+    cfg = mid_cfg()
+    w = _fake_weights()
+    E = cfg.num_experts
+    assert _call_ep(lib, cfg, w, 0, E, T=0) == _abi.MOE_OK
+    assert _call_ep(lib, cfg, w, -1, 4) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_ep(lib, cfg, w, 0, E + 1) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_ep(lib, cfg, w, 5, 4) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_ep(lib, cfg, w, 0, E, out=None) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_ep(lib, cfg, w, 0, E, ws=None) == _abi.MOE_ERR_WORKSPACE
+    # local experts need weights, an empty range does not
+    assert _call_ep(lib, cfg, _fake_weights(w_gate_up=None), 0, 4) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_ep(lib, cfg, _fake_weights(w_gate_up=None, w_down=None), 4, 4, T=0) == _abi.MOE_OK

@@ -349,3 +349,41 @@ def test_generator_is_deterministic():
         assert torch.equal(getattr(a, name), getattr(b, name)), name
     c = moe_inputs.make_layer(CONFIGS["tiny"], seed=1)
     assert not torch.equal(a.x, c.x)
+
+
+# ------------------------------------------------- expert parallelism ----
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_partials_over_a_partition_add_up_to_the_layer(tiny_layer, tiny_result, world):
+    """Expert ranges partitioning [0, E) and shared-feature slices partitioning
+    [0, I_s): the ranks' partial sums add up to the layer output (the one
+    all-reduce of glm5next §One all-reduce)."""
+    cfg = tiny_layer.cfg
+    # plain index arithmetic for the partition (independent of any product helper)
+    e_cuts = [round(i * cfg.E / world) for i in range(world + 1)]
+    s_cuts = [8 * round(i * (cfg.I_s // 8) / world) for i in range(world + 1)]
+    total = torch.zeros_like(tiny_result.out)
+    for r in range(world):
+        total += oracle.moe_partial(tiny_layer, e_cuts[r], e_cuts[r + 1], s_cuts[r], s_cuts[r + 1])
+    assert torch.allclose(total, tiny_result.out, rtol=1e-12, atol=1e-12)
+
+
+def test_partial_of_everything_is_the_layer_and_of_nothing_is_zero(tiny_layer, tiny_result):
+    cfg = tiny_layer.cfg
+    assert torch.allclose(oracle.moe_partial(tiny_layer, 0, cfg.E, 0, cfg.I_s), tiny_result.out, rtol=1e-12,
+                          atol=1e-12)
+    assert torch.count_nonzero(oracle.moe_partial(tiny_layer, 3, 3, 16, 16)) == 0
+
+
+def test_hand_layer_partials(hand):
+    """The one-token hand layer: expert 0's rank holds 0.5*y0, expert 1's
+    s1*y1, the shared slice holds [s1, s1] (closed forms of the layer's
+    worked output: out = [s1, s1] + 0.5 [3 s1, -6 s1] + s1 [s1, s1])."""
+    lay = _hand_layer(hand)
+    s1 = _s(1.0)
+    p0 = oracle.moe_partial(lay, 0, 1, 0, 0)[0].tolist()
+    p1 = oracle.moe_partial(lay, 1, 4, 0, 0)[0].tolist()
+    ps = oracle.moe_partial(lay, 4, 4, 0, 1)[0].tolist()
+    assert p0 == pytest.approx([1.5 * s1, -3.0 * s1], abs=1e-14)
+    assert p1 == pytest.approx([s1 * s1, s1 * s1], abs=1e-14)
+    assert ps == pytest.approx([s1, s1], abs=1e-14)

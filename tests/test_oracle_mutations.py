@@ -173,3 +173,28 @@ def test_override_without_renorm_is_caught(monkeypatch, hand):
 
 
 hand = pins.hand
+
+
+def test_partial_with_inclusive_range_is_caught(monkeypatch, tiny_layer, tiny_result):
+    orig = om.moe_partial
+
+    def inclusive(layer, b, e, s0, s1, **kw):        # the range's end expert counted too
+        return orig(layer, b, min(e + 1, layer.cfg.E), s0, s1, **kw)
+    _patch(monkeypatch, "moe_partial", inclusive)
+    _expect_fail(pins.test_partials_over_a_partition_add_up_to_the_layer, tiny_layer, tiny_result, 2)
+
+
+def test_partial_with_scaled_shared_slice_is_caught(monkeypatch, tiny_layer, tiny_result):
+    orig = om.moe_partial
+
+    def scaled(layer, b, e, s0, s1, **kw):           # shared slice divided by the rank count
+        p = orig(layer, b, e, s0, s1, **kw)
+        if s1 > s0:
+            p = p - 0.5 * orig(layer, b, b, s0, s1, **kw)
+        return p
+    _patch(monkeypatch, "moe_partial", scaled)
+    _expect_fail(pins.test_partials_over_a_partition_add_up_to_the_layer, tiny_layer, tiny_result, 2)
+
+
+tiny_layer = pins.tiny_layer
+tiny_result = pins.tiny_result
