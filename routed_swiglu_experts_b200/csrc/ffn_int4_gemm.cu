@@ -9,16 +9,23 @@
 //   down:     y[t, n] = bf16( row_scale[t] * sum_i W_d[n, i] h[t, i] )
 //
 // Same tile and roles as the bf16 CTA-pair kernel (weights = M, 256 rows per
-// pair; tokens = N rounded to 16; two 256-column TMEM accumulators), plus
-// four dequantisation warps per CTA: TMA copies the int4 codes of the CTA's
-// 128 weight rows (32 bytes per row per 64-deep K step) into a staging ring;
-// each dequantisation thread turns one row's 64 codes into fp16 weights
+// pair; tokens = N rounded to 16; two 256-column TMEM accumulators), plus a
+// code producer and eight dequantisation warps per CTA: TMA copies the int4
+// codes of the CTA's 128 weight rows (128 bytes per row: four 64-deep K
+// steps per copy) into a two-stage staging ring; two threads per weight row
+// turn its 32 codes per K step into fp16 weights
 //   (q - 8) * scale   -- exact in fp16: a 4-bit integer times a bf16 scale
-// and writes them, 128-byte swizzled, into the MMA's A stage, then the warp
-// arrives on the pair's full barrier.  Within every aligned 8 of K the
-// weights sit in the order {0, 4, 1, 5, 2, 6, 3, 7} (how four LOP3s split a
-// 32-bit code word); the tokens are prepared in the same order, and the
-// gate/up epilogue writes h in it, so the K sum is unchanged.
+// (within the fp16 range moe.h states for the W4A16 format) and write them,
+// 128-byte swizzled, into the MMA's A stage, then each warp arrives on the
+// pair's full barrier.  The code-to-fp16 step is the exponent-OR ("magic
+// number") conversion of mixed-input GEMM kernels -- OR a nibble into the
+// mantissa of fp16 1024.0, subtract 1024 + 8 -- as described by Kim et al.,
+// "Who Says Elephants Can't Run: Bringing Large Scale MoE Models into Cloud
+// Scale Production" (2022), and used by the Marlin kernels (Frantar et al.,
+// 2024).  Within every aligned 8 of K the weights sit in the order
+// {0, 4, 1, 5, 2, 6, 3, 7} (how four LOP3s split a 32-bit code word); the
+// tokens are prepared in the same order, and the gate/up epilogue writes h
+// in it, so the K sum is unchanged.
 // Tiles are handed out from a queue in the workspace header as in the bf16
 // kernel.  Every mbarrier wait is bounded (MOE_ERR_DEVICE_TIMEOUT on expiry).
 #include <cstring>

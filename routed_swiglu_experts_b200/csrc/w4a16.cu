@@ -9,9 +9,12 @@
 // Weight format: uint8 [N, K/2], the code of k = 2c in the low nibble of byte
 // c and k = 2c+1 in the high nibble; w = (code - 8) * scale[n, k / 128].
 //
-// Dequantisation.  For a 32-bit word w of 8 codes (nibble i = physical
-// offset i), OR-ing the fp16 exponent of 1024 and subtracting the offset
-// with one sub.f16x2 gives exact fp16 pairs:
+// Dequantisation: the exponent-OR ("magic number") integer-to-fp16
+// conversion of mixed-input GEMM kernels (Kim et al., "Who Says Elephants
+// Can't Run: Bringing Large Scale MoE Models into Cloud Scale Production",
+// 2022; the Marlin kernels, Frantar et al., 2024).  For a 32-bit word w of 8
+// codes (nibble i = physical offset i), OR-ing the fp16 exponent of 1024 and
+// subtracting the offset with one sub.f16x2 gives exact fp16 pairs:
 //   P0 = ((w      & 0x000F000F) | 0x64006400) - 1032 = {q0 - 8,       q4 - 8}
 //   P1 = ((w      & 0x00F000F0) | 0x64006400) - 1152 = {16 (q1 - 8),  16 (q5 - 8)}
 //   P2 = ((w >> 8 & 0x000F000F) | 0x64006400) - 1032 = {q2 - 8,       q6 - 8}
