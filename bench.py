@@ -218,11 +218,10 @@ def w4a16_bytes(cfg, ids):
 
 def launches_per_step(cfg):
     """Kernels one forward launches: router 3 (weight split, tensor-core
-    logits, top-k; for T <= 64 tokens 2: fp64 logits, top-k), permute 2
-    (count/rank with the scan in its last block, scatter), combine 1, plus
-    the expert FFN path and the shared expert's launches when it does not
-    ride in the routed ones."""
-    n = (2 if cfg.T <= 64 else 3) + 3
+    logits, top-k), permute 2 (count/rank with the scan in its last block,
+    scatter), combine 1, plus the expert FFN path and the shared expert's
+    launches when it does not ride in the routed ones."""
+    n = 6
     prefill = cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E   # int4 dequantised in shared memory, tensor cores
     gemv = cfg.w4a16 and not prefill                      # int4 dequantised in registers
     shared = 0

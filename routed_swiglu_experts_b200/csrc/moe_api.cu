@@ -148,12 +148,10 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
       // down projection's activations are prepared
       float* gu = at<float>(ws, L.h);
       float* gu_s = shared_in_gemv ? at<float>(ws, L.small_part) : nullptr;
-      float* corr = at<float>(ws, L.corr);
-      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, corr, gu,
-                                       shared_in_gemv ? x_shared : nullptr, T, gu_s, stream));
+      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, shared_in_gemv ? x_shared : nullptr, T,
+                                       gu_s, stream));
       if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
-      MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, corr, w_perm, y_perm, gu_s, T, hs, shared_out,
-                                     stream));
+      MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, gu_s, T, hs, shared_out, stream));
     }
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, qd, sms, stream));
   }
@@ -209,7 +207,6 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.shared_out = take(T * H * 2);
   const size_t kmax = std::max(H, I);
   L.act16 = take(int4 ? R * kmax * 2 : 0);
-  L.corr = take(int4 ? R * (kmax / 128) * 4 : 0);
   L.small_part = take(Is > 0 ? dense_small_part_floats(static_cast<int>(H), static_cast<int>(Is)) * sizeof(float) : 0);
   L.total = off;
   return L;

@@ -32,10 +32,6 @@ struct RouterPlan {
   int ks;  // k-splits of the logits GEMM (partials summed by the top-k kernel)
 };
 RouterPlan router_plan(int T, int E, int H, int num_sms);
-// At most this many tokens: the router computes fp64 logits directly (no
-// weight split, no tensor cores, no near-tie re-rank needed).
-constexpr int kRouterF64MaxTokens = 64;
-bool router_f64_preferred(int T);
 size_t router_partial_floats(int Tmax, int E);
 size_t router_topk_smem(int E);
 // Split-K tensor-core GEMM with fp32 partials part[s][rows][N] over `parts`
@@ -102,13 +98,12 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
 // the down projection's activation prep, and down into shared_out.
 constexpr int kW4a16SharedMaxTokens = 32;
 bool w4a16_shared_fusable(int T, int Is);
-// corr: scratch [rows, max(H, I) / 128] fp32 (per row and 128-wide group).
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* corr, float* gu,
-                                const void* x_shared, int T, float* gu_shared, cudaStream_t stream);
+                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
+                                int T, float* gu_shared, cudaStream_t stream);
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
-                              int rows, void* act16, float* corr, const float* w_perm, void* y_perm,
-                              const float* gu_shared, int T, void* h_shared, void* shared_out, cudaStream_t stream);
+                              int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
+                              int T, void* h_shared, void* shared_out, cudaStream_t stream);
 
 // W4A16 grouped GEMMs for many tokens per expert: int4 codes dequantised to
 // fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.
@@ -131,7 +126,7 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
 // Workspace layout (byte offsets from the workspace base; 256-aligned).
 struct WsLayout {
   size_t header, logits, w_split, ids, wts, offsets, row_of, src, w_perm, block_base, local_rank;
-  size_t x_perm, h, h_shared, y_perm, shared_out, act16, corr, small_part, total;
+  size_t x_perm, h, h_shared, y_perm, shared_out, act16, small_part, total;
 };
 WsLayout ws_layout(const moe_config& cfg, int Tmax);
 

@@ -443,112 +443,6 @@ size_t rows_smem(int E, int tb) {
   return kRowsWarps * rows_scratch_per_warp(E) + 2 * static_cast<size_t>(tb) * E * sizeof(float);
 }
 
-// ------------------------------------------------ few tokens: fp64 router --
-// For a handful of tokens (decode) the router is a small GEMV whose cost is
-// reading the fp32 weight once; the tensor-core path's weight split, split-K
-// partials and near-tie re-rank cost far more than the arithmetic.  Here the
-// logits are computed directly in fp64 (every bf16 x fp32 product is exact in
-// fp64, and the fp64 sum is exact to ~1e-16 relative), so the selection is
-// the exact-arithmetic one without any re-rank, and the weights are the fp64
-// scores rounded to fp32.
-
-constexpr int kF64Warps = 8;   // experts per block (one per warp)
-constexpr int kF64Tok = 8;     // tokens per warp
-
-// logit64[t][e] = sum_h x[t, h] * w[e, h] in fp64.  Grid (ceil(E / 8),
-// ceil(T / 8)); warp w: expert blockIdx.x * 8 + w, tokens blockIdx.y * 8 ..
-// + 7; each lane sums h = 4 lane + 128 i (sequentially), then a fixed
-// xor-shuffle tree: deterministic.
-__global__ void __launch_bounds__(kF64Warps * 32)
-    router_logits_f64_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, int T, int E, int H,
-                             double* __restrict__ logit64) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int e = blockIdx.x * kF64Warps + warp;
-  const int t0 = blockIdx.y * kF64Tok;
-  if (e >= E) return;
-  double acc[kF64Tok];
-#pragma unroll
-  for (int j = 0; j < kF64Tok; ++j) acc[j] = 0.0;
-  const float* wrow = wr + static_cast<size_t>(e) * H;
-  for (int h = 4 * lane; h < H; h += 128) {
-    const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + h));
-#pragma unroll
-    for (int j = 0; j < kF64Tok; ++j) {
-      if (t0 + j < T) {
-        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(x + static_cast<size_t>(t0 + j) * H + h));
-        acc[j] = fma(static_cast<double>(bf16lo(xv.x)), static_cast<double>(wv.x), acc[j]);
-        acc[j] = fma(static_cast<double>(bf16hi(xv.x)), static_cast<double>(wv.y), acc[j]);
-        acc[j] = fma(static_cast<double>(bf16lo(xv.y)), static_cast<double>(wv.z), acc[j]);
-        acc[j] = fma(static_cast<double>(bf16hi(xv.y)), static_cast<double>(wv.w), acc[j]);
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kF64Tok; ++j) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int j = 0; j < kF64Tok; ++j)
-      if (t0 + j < T) logit64[static_cast<size_t>(t0 + j) * E + e] = acc[j];
-  }
-}
-
-// One warp per token: s = sigmoid(logit) and b = s + bias in fp64, the k
-// largest b in (b desc, id asc) order by k warp-wide argmax rounds, the
-// weights alpha * s (renormalised over the k first if asked; fp64, rounded
-// to fp32 at the end).  dynamic smem: kF64Warps x (b[E], s[E]) fp64.
-__global__ void __launch_bounds__(kF64Warps * 32)
-    router_topk_f64_kernel(const double* __restrict__ logit64, const float* __restrict__ bias, int T, int E, int k,
-                           float alpha, int renorm, int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x * kF64Warps + warp;
-  if (t >= T) return;
-  double* b64 = reinterpret_cast<double*>(smem_raw) + static_cast<size_t>(warp) * 2 * E;
-  double* s64 = b64 + E;
-  for (int e = lane; e < E; e += 32) {
-    const double s = 1.0 / (1.0 + exp(-logit64[static_cast<size_t>(t) * E + e]));
-    s64[e] = s;
-    b64[e] = s + (bias != nullptr ? static_cast<double>(bias[e]) : 0.0);
-  }
-  __syncwarp();
-  const int nm = (E + 31) / 32;
-  uint32_t taken = 0;
-  int my_id = 0;        // lane j < k keeps the j-th selected expert
-  double my_s = 0.0;
-  double wsum = 0.0;
-  for (int r = 0; r < k; ++r) {
-    double v = -INFINITY;
-    int id = 0x7fffffff;
-    for (int m = 0; m < nm; ++m) {
-      const int e = lane + 32 * m;
-      if (e < E && !((taken >> m) & 1u)) {
-        const double bv = b64[e];
-        if (bv > v || (bv == v && e < id)) {
-          v = bv;
-          id = e;
-        }
-      }
-    }
-    warp_argmax(v, id);
-    if ((id & 31) == lane) taken |= 1u << (id / 32);
-    const double sv = s64[id];
-    wsum += sv;
-    if (lane == r) {
-      my_id = id;
-      my_s = sv;
-    }
-  }
-  if (lane < k) {
-    const size_t o = static_cast<size_t>(t) * k + lane;
-    ids_out[o] = my_id;
-    w_out[o] = static_cast<float>(renorm ? (my_s / wsum) * static_cast<double>(alpha)
-                                         : my_s * static_cast<double>(alpha));
-  }
-}
-
 }  // namespace
 
 RouterPlan router_plan(int T, int E, int H, int num_sms) {
@@ -570,26 +464,9 @@ size_t router_partial_floats(int Tmax, int E) {
 
 size_t router_topk_smem(int E) { return topk_smem_per_warp(E); }
 
-bool router_f64_preferred(int T) { return T <= kRouterF64MaxTokens; }
-
 cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const void* x, int T, int32_t* ids,
                           float* wts, float* part, void* w_split, int32_t* err, int num_sms, cudaStream_t stream) {
   const int E = cfg.num_experts, H = cfg.hidden, k = cfg.top_k;
-  if (router_f64_preferred(T)) {
-    double* logit64 = reinterpret_cast<double*>(part);  // T x E doubles: far inside the partials region
-    const dim3 grid((E + kF64Warps - 1) / kF64Warps, (T + kF64Tok - 1) / kF64Tok);
-    router_logits_f64_kernel<<<grid, kF64Warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), w.router_w,
-                                                                  T, E, H, logit64);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t smem = static_cast<size_t>(kF64Warps) * 2 * E * sizeof(double);
-    e = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_f64_kernel),
-                         static_cast<int>(kF64Warps * 2 * MOE_MAX_EXPERTS * sizeof(double)));
-    if (e != cudaSuccess) return e;
-    router_topk_f64_kernel<<<(T + kF64Warps - 1) / kF64Warps, kF64Warps * 32, smem, stream>>>(
-        logit64, w.correction_bias, T, E, k, cfg.routed_scaling_factor, cfg.renormalize, ids, wts);
-    return cudaGetLastError();
-  }
   const RouterPlan p = router_plan(T, E, H, num_sms);
   const int n4 = E * H / 4;
   router_split_kernel<<<(n4 + 255) / 256, 256, 0, stream>>>(reinterpret_cast<const float4*>(w.router_w), n4,

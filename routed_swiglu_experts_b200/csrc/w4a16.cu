@@ -57,45 +57,14 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-#ifndef MOE_W4A16_FOLD
-#define MOE_W4A16_FOLD 0
-#endif
 __device__ __forceinline__ Pairs code_pairs(uint32_t w) {
   const uint32_t w8 = w >> 8;
   Pairs r;
-#if MOE_W4A16_FOLD
-  // biased values 1024 + q (even nibbles) and 1024 + 16 q (odd); the offsets
-  // 1032 and 1152 are taken off once per (token, group) after the MMAs
-  r.p0 = (w & 0x000F000Fu) | 0x64006400u;
-  r.p1 = (w & 0x00F000F0u) | 0x64006400u;
-  r.p2 = (w8 & 0x000F000Fu) | 0x64006400u;
-  r.p3 = (w8 & 0x00F000F0u) | 0x64006400u;
-#else
   r.p0 = hsub2((w & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // - {1032, 1032}
   r.p1 = hsub2((w & 0x00F000F0u) | 0x64006400u, 0x64806480u);   // - {1152, 1152}
   r.p2 = hsub2((w8 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
   r.p3 = hsub2((w8 & 0x00F000F0u) | 0x64006400u, 0x64806480u);
-#endif
   return r;
-}
-
-// Per (activation row, 128-wide group) correction for the biased codes:
-// the MMA of biased codes with the slot-ordered activations a exceeds the
-// wanted sum by 1032 * (sum of a in even-nibble slots) + 1152 * (sum in
-// odd-nibble slots, which hold x / 16): subtracting it leaves
-// sum_k (q_k - 8) x_k.  `p` is one thread's share over its 8 values; the 16
-// threads of a group (consecutive lanes) add theirs in a fixed tree.
-__device__ __forceinline__ float group_offset_share(uint4 o) {
-  const __half2 a04 = *reinterpret_cast<const __half2*>(&o.x), b15 = *reinterpret_cast<const __half2*>(&o.y);
-  const __half2 a26 = *reinterpret_cast<const __half2*>(&o.z), b37 = *reinterpret_cast<const __half2*>(&o.w);
-  const float2 f04 = __half22float2(a04), f15 = __half22float2(b15), f26 = __half22float2(a26),
-               f37 = __half22float2(b37);
-  return 1032.f * ((f04.x + f04.y) + (f26.x + f26.y)) + 1152.f * ((f15.x + f15.y) + (f37.x + f37.y));
-}
-__device__ __forceinline__ float sum16(float p) {
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-  return p;
 }
 
 // One 128-wide group, one m16 tile (rows g and g+8 of the tile): 8 MMAs.
@@ -118,16 +87,10 @@ __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) { return __bflo
 // Activations in MMA slot order.  One thread per 8 consecutive values of a
 // row: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16}.
 __global__ void __launch_bounds__(256)
-    w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, long long n8, uint4* __restrict__ act16,
-                      float* __restrict__ corr) {
+    w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, long long n8, uint4* __restrict__ act16) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-#if MOE_W4A16_FOLD
-  // n8 is a multiple of 16 (K % 128 == 0): a group's 16 threads are all in or all out
-  const uint4 v = idx < n8 ? __ldg(reinterpret_cast<const uint4*>(act) + idx) : make_uint4(0, 0, 0, 0);
-#else
   if (idx >= n8) return;
   const uint4 v = __ldg(reinterpret_cast<const uint4*>(act) + idx);
-#endif
   const __half2 a04 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));
   const __half2 b15 = __floats2half2_rn(bf16hi(v.x) * 0.0625f, bf16hi(v.z) * 0.0625f);
   const __half2 a26 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));
@@ -137,11 +100,6 @@ __global__ void __launch_bounds__(256)
   o.y = *reinterpret_cast<const uint32_t*>(&b15);
   o.z = *reinterpret_cast<const uint32_t*>(&a26);
   o.w = *reinterpret_cast<const uint32_t*>(&b37);
-#if MOE_W4A16_FOLD
-  const float c = sum16(group_offset_share(o));
-  if (idx >= n8) return;
-  if ((idx & 15) == 0) corr[idx >> 4] = c;
-#endif
   act16[idx] = o;
 }
 
@@ -159,10 +117,28 @@ __device__ __forceinline__ float swiglu_clamped_f(float g, float u, float L) {
   return __fdividef(gc, 1.f + __expf(-gc)) * uc;
 }
 
-// Eight consecutive features of routed row r (idx = r * I / 8 + f / 8): the
-// clamped SwiGLU of the fp32 gate/up, rounded to bf16 like the bf16 path's h,
-// in MMA slot order as fp16.
-__device__ __forceinline__ uint4 swiglu_slot_order(const float* __restrict__ gu, int I, long long idx, float L) {
+__global__ void __launch_bounds__(256)
+    w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
+                             const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs) {
+  long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n8) {
+    idx -= n8;
+    if (gus == nullptr || idx >= n8s) return;
+    const int is8 = Is / 8;
+    const long long r = idx / is8;
+    const int f = static_cast<int>(idx - r * is8) * 8;
+    const float* gp = gus + r * 2 * Is + f;
+    float h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = swiglu_clamped_f(__ldg(gp + j), __ldg(gp + Is + j), L);
+    uint4 o;
+    o.x = pack_bf16x2(h[0], h[1]);
+    o.y = pack_bf16x2(h[2], h[3]);
+    o.z = pack_bf16x2(h[4], h[5]);
+    o.w = pack_bf16x2(h[6], h[7]);
+    *reinterpret_cast<uint4*>(hs + r * Is + f) = o;
+    return;
+  }
   const int i8 = I / 8;
   const long long r = idx / i8;
   const int f = static_cast<int>(idx - r * i8) * 8;
@@ -183,48 +159,7 @@ __device__ __forceinline__ uint4 swiglu_slot_order(const float* __restrict__ gu,
   o.y = *reinterpret_cast<const uint32_t*>(&b15);
   o.z = *reinterpret_cast<const uint32_t*>(&a26);
   o.w = *reinterpret_cast<const uint32_t*>(&b37);
-  return o;
-}
-
-__global__ void __launch_bounds__(256)
-    w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
-                             const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs,
-                             float* __restrict__ corr) {
-  long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-#if MOE_W4A16_FOLD
-  // the routed rows' group corrections need all 16 lanes of a group; a warp
-  // holds whole groups (n8 % 16 == 0), so the routed lanes of a warp reduce
-  // among themselves before any lane takes the shared-expert branch
-  if (idx < n8 || (idx - (idx & 31)) < n8) {
-    uint4 o = make_uint4(0, 0, 0, 0);
-    if (idx < n8) o = swiglu_slot_order(gu, I, idx, L);
-    const float c = sum16(group_offset_share(o));
-    if (idx < n8) {
-      if ((idx & 15) == 0) corr[idx >> 4] = c;
-      act16[idx] = o;
-      return;
-    }
-  }
-#endif
-  if (idx >= n8) {
-    idx -= n8;
-    if (gus == nullptr || idx >= n8s) return;
-    const int is8 = Is / 8;
-    const long long r = idx / is8;
-    const int f = static_cast<int>(idx - r * is8) * 8;
-    const float* gp = gus + r * 2 * Is + f;
-    float h[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) h[j] = swiglu_clamped_f(__ldg(gp + j), __ldg(gp + Is + j), L);
-    uint4 o;
-    o.x = pack_bf16x2(h[0], h[1]);
-    o.y = pack_bf16x2(h[2], h[3]);
-    o.z = pack_bf16x2(h[4], h[5]);
-    o.w = pack_bf16x2(h[6], h[7]);
-    *reinterpret_cast<uint4*>(hs + r * Is + f) = o;
-    return;
-  }
-  act16[idx] = swiglu_slot_order(gu, I, idx, L);
+  act16[idx] = o;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -335,8 +270,7 @@ template <bool F32OUT>
 __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
     w4a16_gemv_kernel(const uint4* __restrict__ act16, const int32_t* __restrict__ offsets,
                       const uint8_t* __restrict__ q, const __nv_bfloat16* __restrict__ scales, int N, int K,
-                      const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj,
-                      const float* __restrict__ corr) {
+                      const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj) {
   extern __shared__ uint4 gemv_ring[];
   constexpr int S = kGemvStages;
   // blocks of the first grid row take the shared expert (when there is one):
@@ -376,11 +310,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
     const int ntok = min(kTok, r_end - tc);
     const bool has = g < ntok;
     const uint4* ap = act16 + static_cast<size_t>(tc + (has ? g : 0)) * (K / 8) + 4 * t;
-#if MOE_W4A16_FOLD
-    // group corrections of this thread's two token columns (2t, 2t + 1)
-    const float* cr0 = corr + static_cast<size_t>(tc + min(2 * t, ntok - 1)) * groups;
-    const float* cr1 = corr + static_cast<size_t>(tc + min(2 * t + 1, ntok - 1)) * groups;
-#endif
 #pragma unroll
     for (int i = 0; i < S - 1; ++i) {
       if (i < groups) issue(q0, i, i);
@@ -421,15 +350,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
           const uint4 c0 = st[0], c8 = st[32];
           float tt[4] = {0.f, 0.f, 0.f, 0.f};
           tile_group(tt, c0, c8, act);
-#if MOE_W4A16_FOLD
-          {
-            const float k0 = __ldg(cr0 + gq), k1 = __ldg(cr1 + gq);
-            tt[0] -= k0;
-            tt[1] -= k1;
-            tt[2] -= k0;
-            tt[3] -= k1;
-          }
-#endif
           float a0, a8;
           if (batch8) {
             const uint32_t w0 = (jj >> 1) == 0 ? sv0.x : (jj >> 1) == 1 ? sv0.y : (jj >> 1) == 2 ? sv0.z : sv0.w;
@@ -466,23 +386,23 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
   }
 }
 
-cudaError_t launch_prep(const void* act, int rows, int K, void* act16, float* corr, cudaStream_t stream) {
+cudaError_t launch_prep(const void* act, int rows, int K, void* act16, cudaStream_t stream) {
   const long long n8 = static_cast<long long>(rows) * (K / 8);
   w4a16_prep_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(act), n8, static_cast<uint4*>(act16), corr);
+      static_cast<const __nv_bfloat16*>(act), n8, static_cast<uint4*>(act16));
   return cudaGetLastError();
 }
 
 template <bool F32OUT>
 cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, const void* act16,
                         const int32_t* offsets, const float* w_perm, void* out, const SharedJob& sj,
-                        const float* corr, cudaStream_t stream) {
+                        cudaStream_t stream) {
   const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
   const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
   if (grid.y == 0) return cudaSuccess;  // no routed expert and no shared expert in this call
   w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, kGemvSmem, stream>>>(
       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
-      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj, corr);
+      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
   return cudaGetLastError();
 }
 
@@ -491,29 +411,29 @@ cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, 
 bool w4a16_shared_fusable(int T, int Is) { return Is > 0 && T >= 1 && T <= kW4a16SharedMaxTokens; }
 
 cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* corr, float* gu,
-                                const void* x_shared, int T, float* gu_shared, cudaStream_t stream) {
+                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
+                                int T, float* gu_shared, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
-  cudaError_t e = launch_prep(x_perm, rows, H, act16, corr, stream);
+  cudaError_t e = launch_prep(x_perm, rows, H, act16, stream);
   if (e != cudaSuccess) return e;
   SharedJob sj{};
   if (x_shared != nullptr)  // shared gate/up [2 I_s, H] x tokens [T, H] -> fp32 [T, 2 I_s]
     sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_gate_up), static_cast<const __nv_bfloat16*>(x_shared),
                    gu_shared, 2 * cfg.shared_inter, H, T};
   // W_gu [E, 2I, H/2]: one matrix of 2I rows per expert (gate rows, then up rows)
-  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, sj, corr, stream);
+  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, sj, stream);
 }
 
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
-                              int rows, void* act16, float* corr, const float* w_perm, void* y_perm,
-                              const float* gu_shared, int T, void* h_shared, void* shared_out, cudaStream_t stream) {
+                              int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
+                              int T, void* h_shared, void* shared_out, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts, Is = cfg.shared_inter;
   const long long n8 = static_cast<long long>(rows) * (I / 8);
   const long long n8s = gu_shared != nullptr ? static_cast<long long>(T) * (Is / 8) : 0;
   if (n8 + n8s > 0) {
     w4a16_prep_swiglu_kernel<<<static_cast<unsigned>((n8 + n8s + 255) / 256), 256, 0, stream>>>(
         gu, I, n8, cfg.swiglu_limit, static_cast<uint4*>(act16), gu_shared, Is, n8s,
-        static_cast<__nv_bfloat16*>(h_shared), corr);
+        static_cast<__nv_bfloat16*>(h_shared));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -521,7 +441,7 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
   if (gu_shared != nullptr)  // shared down [H, I_s] x h_s [T, I_s] -> bf16 [T, H], unscaled
     sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_down), static_cast<const __nv_bfloat16*>(h_shared),
                    shared_out, H, Is, T};
-  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, sj, corr, stream);
+  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, sj, stream);
 }
 
 }  // namespace moe

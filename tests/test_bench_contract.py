@@ -30,9 +30,8 @@ def test_gemm_flops_of_the_mid_layer():
     # gate/up + down (shared expert as a second problem), combine
     ("mid", 8),
     ("large_prefill", 8),
-    # fp64 router (logits + top-k) for 32 tokens, ... + W4A16 (prep + GEMV) x 2,
-    # the shared expert inside the GEMV launches
-    ("decode_w4a16", 9),
+    # ... + W4A16 (prep + GEMV) x 2, the shared expert inside the GEMV launches
+    ("decode_w4a16", 10),
     # ... + token prep + dequantising gate/up and down + bf16 shared gate/up
     # and down launches
     ("prefill_w4a16", 11),
