@@ -67,9 +67,18 @@ constexpr uint32_t kTileReaders = 1 + 4 + 1 + 4;
 
 enum class Kind { GateUp, Down };
 
+// Token boxes of 128, 64, 32, 16 and 8 rows: each CTA of a pair copies the
+// smallest box that holds its nmma / 2 token rows, so a ragged last tile of
+// an expert moves fewer bytes through L2 into shared memory (one copy per
+// chunk either way).
+constexpr int kTokBoxes = 5;
+__host__ __device__ constexpr int tok_box_index(int rows_per_cta) {
+  return rows_per_cta > 64 ? 0 : rows_per_cta > 32 ? 1 : rows_per_cta > 16 ? 2 : rows_per_cta > 8 ? 3 : 4;
+}
+
 struct alignas(64) PairParams {
   CUtensorMap tma_w[2];       // weights: gate/up {K, 8, 2, N/8, G} box {64, 8, 2, 8, 1}; down {K, N, G} box {64, 128, 1}
-  CUtensorMap tma_x[2];       // tokens {K, rows} box {64, 128}
+  CUtensorMap tma_x[2][kTokBoxes];  // tokens {K, rows} box {64, 128 >> i}: a tile copies only the rows it uses
   const int32_t* offsets[2];  // grouped problem: [groups+1]; else nullptr
   __nv_bfloat16* out[2];      // [rows, N]
   const float* row_scale[2];  // down: per token row (or nullptr)
@@ -187,7 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 4 && lane == 0) {
     for (int p = 0; p < P.nprob; ++p) {
       tma_prefetch_desc(&P.tma_w[p]);
-      tma_prefetch_desc(&P.tma_x[p]);
+      for (int b = 0; b < kTokBoxes; ++b) tma_prefetch_desc(&P.tma_x[p][b]);
     }
   }
   if (warp == 0) {  // per-problem tile counts; grouped problems: offsets + token-tile prefix
@@ -294,6 +303,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int nkb = P.k_blocks[p];
         const int nstage = (nkb + KCH - 1) / KCH;  // the last stage of an odd count holds one chunk
         const int kpre = nstage > 2 ? nstage - 2 : 0;
+        const int xb = tok_box_index(ti.nmma / 2);
+        const uint32_t b_bytes = static_cast<uint32_t>((TOK / 2) >> xb) * BK * 2;  // this CTA's token copy per chunk
         for (int st = 0; st < nstage; ++st) {
           if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns)) {
             fail(31);
@@ -301,7 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             break;
           }
           const int nk = min(KCH, nkb - st * KCH);
-          if (leader) mbar_arrive_expect_tx(&c.full[stage], 2u * static_cast<uint32_t>(nk * (A_BYTES + B_BYTES)));
+          if (leader) mbar_arrive_expect_tx(&c.full[stage], 2u * static_cast<uint32_t>(nk) * (A_BYTES + b_bytes));
           const uint32_t bar = leader_bar(&c.full[stage]);
           for (int ch = 0; ch < nk; ++ch) {
             const int kc = (st * KCH + ch) * BK;
@@ -313,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
               tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
             }
-            tma_load_2d_pair(smem_b + stage * B_STAGE + ch * B_BYTES, &P.tma_x[p], kc, xrow, bar);
+            tma_load_2d_pair(smem_b + stage * B_STAGE + ch * B_BYTES, &P.tma_x[p][xb], kc, xrow, bar);
           }
           if (leader && st == kpre) t_next = atomicAdd(P.queue, 1);
           ++issued;
@@ -561,11 +572,15 @@ bool encode_w_gu(CUtensorMap* m, const void* base, int groups, int N, int K) {
   return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-bool encode_x(CUtensorMap* m, const void* base, int rows, int K) {
+bool encode_x(CUtensorMap (&m)[kTokBoxes], const void* base, int rows, int K) {
   const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {BK, TOK / 2};
-  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  for (int b = 0; b < kTokBoxes; ++b) {
+    const uint32_t box[2] = {BK, static_cast<uint32_t>((TOK / 2) >> b)};
+    if (!encode_tma(&m[b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  return true;
 }
 
 // CTA pairs that can be resident at once on the current device (a pair must
@@ -607,7 +622,7 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
     return cudaErrorInvalidValue;  // one grouped problem per launch (one offsets table in shared memory)
   for (int i = 0; i < np; ++i) {
     const FfnProblem& f = *probs[i];
-    if (!encode_x(&P.tma_x[i], f.a, f.rows, f.K)) return cudaErrorInvalidValue;
+    if (!encode_x(P.tma_x[i], f.a, f.rows, f.K)) return cudaErrorInvalidValue;
     const bool okw = KIND == Kind::GateUp ? encode_w_gu(&P.tma_w[i], f.w, f.groups, f.N, f.K)
                                           : encode_w(&P.tma_w[i], f.w, f.groups, f.N, f.K, 128);
     if (!okw) return cudaErrorInvalidValue;
@@ -651,7 +666,7 @@ cudaError_t launch_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* q
   void* h = base + 20480;  // bf16 [16, 64]
   PairParams P;
   memset(&P, 0, sizeof(P));
-  if (!encode_x(&P.tma_x[0], x, 16, 64) || !encode_w_gu(&P.tma_w[0], w, 1, 64, 64)) return cudaErrorInvalidValue;
+  if (!encode_x(P.tma_x[0], x, 16, 64) || !encode_w_gu(&P.tma_w[0], w, 1, 64, 64)) return cudaErrorInvalidValue;
   P.offsets[0] = nullptr;
   P.out[0] = static_cast<__nv_bfloat16*>(h);
   P.groups[0] = 1;
