@@ -207,8 +207,8 @@ def run_cpu_baseline(inp, min_seconds=10.0, max_passes=20, gpu_out=None, gpu_ids
 
 def w4a16_bytes(cfg, ids):
     """HBM bytes the W4A16 expert FFN call must move: codes + scales of every
-    touched expert, the bf16 shared expert, and its activations (x_perm and
-    x read, y_perm and the shared output written)."""
+    touched expert, the bf16 shared expert, and its activations (the T*k
+    gathered token rows and x read, y_perm and the shared output written)."""
     touched = int(len(set(ids.reshape(-1).tolist())))
     per_expert = (2 * cfg.I * cfg.H // 2 + cfg.H * cfg.I // 2) + 2 * (2 * cfg.I * cfg.H // 128 + cfg.H * cfg.I // 128)
     shared = 2 * (2 * cfg.I_s * cfg.H + cfg.H * cfg.I_s)
@@ -219,8 +219,10 @@ def w4a16_bytes(cfg, ids):
 def launches_per_step(cfg):
     """Kernels one forward launches: router 3 (weight split, tensor-core
     logits, top-k), permute 2 (count/rank with the scan in its last block,
-    scatter), combine 1, plus the expert FFN path and the shared expert's
-    launches when it does not ride in the routed ones."""
+    then the scatter into x_perm, or for int4 experts the maps alone, their
+    activation conversion gathering the rows), combine 1, plus the expert
+    FFN path and the shared expert's launches when it does not ride in the
+    routed ones."""
     n = 6
     prefill = cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E   # int4 dequantised in shared memory, tensor cores
     gemv = cfg.w4a16 and not prefill                      # int4 dequantised in registers
@@ -317,15 +319,14 @@ def measure_decode(dev, iters, clocks, max_over_ranks):
     row_of = torch.empty(R, dtype=torch.int32, device=dev)
     src = torch.empty(R, dtype=torch.int32, device=dev)
     w_perm = torch.empty(R, dtype=torch.float32, device=dev)
-    x_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
     y_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
     sh = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     rse.moe_router_topk(layer.cfg, layer.w, x, T, ids, tw, layer.ws)
-    rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
+    rse.moe_permute(layer.cfg, ids, tw, None, T, offs, row_of, src, w_perm, None, layer.ws)
 
-    def ffn():
-        rse.moe_grouped_swiglu_ffn(layer.cfg, layer.w, x_perm, offs, w_perm, T, y_perm, x, sh, layer.ws)
+    def ffn():  # the FFN call moe_forward makes: the permute's gather fused into its loads
+        rse.moe_grouped_swiglu_ffn_gather(layer.cfg, layer.w, x, T, src, offs, w_perm, y_perm, sh, layer.ws)
 
     def fwd():
         layer.forward(x, out=out)
@@ -421,7 +422,9 @@ def bench_ours(args, rank, world, local_rank):
     ms = max_over_ranks(e0.elapsed_time(e1))
     ms_per_step = ms / args.steps
 
-    # --- per-stage durations (same C-ABI calls as the forward, events between)
+    # --- per-stage durations (the kernels the forward launches, one C-ABI call
+    # per stage, events between).  As in moe_forward: bf16 experts permute
+    # into x_perm; int4 experts write the maps only and gather in the FFN.
     T, k, E, H = c.T, c.k, c.E, c.H
     R = T * k
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
@@ -430,7 +433,16 @@ def bench_ours(args, rank, world, local_rank):
     row_of = torch.empty(R, dtype=torch.int32, device=dev)
     src = torch.empty(R, dtype=torch.int32, device=dev)
     w_perm = torch.empty(R, dtype=torch.float32, device=dev)
-    x_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    x_perm = None if c.w4a16 else torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+
+    def permute():
+        rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
+
+    def ffn():
+        if x_perm is None:
+            rse.moe_grouped_swiglu_ffn_gather(layer.cfg, layer.w, x, T, src, offs, w_perm, y_perm, sh, layer.ws)
+        else:
+            rse.moe_grouped_swiglu_ffn(layer.cfg, layer.w, x_perm, offs, w_perm, T, y_perm, x, sh, layer.ws)
     y_perm = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
     sh = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     n_it = max(3, min(args.stage_iters, args.steps))
@@ -443,10 +455,10 @@ def bench_ours(args, rank, world, local_rank):
         rse.moe_router_topk(layer.cfg, layer.w, x, T, ids, tw, layer.ws)
         if ev:
             ev[1].record(stream)
-        rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
+        permute()
         if ev:
             ev[2].record(stream)
-        rse.moe_grouped_swiglu_ffn(layer.cfg, layer.w, x_perm, offs, w_perm, T, y_perm, x, sh, layer.ws)
+        ffn()
         if ev:
             ev[3].record(stream)
         rse.moe_combine(layer.cfg, y_perm, row_of, None, sh, T, out)

@@ -166,12 +166,15 @@ MOE_API moe_status moe_router_topk(const moe_config* cfg, const moe_weights* w,
  * stable counting sort of the slots i = t*k + j by expert id.
  *   topk_ids        int32 [T, k] in (each in [0, E), distinct per token)
  *   topk_w          fp32  [T, k] in
- *   x               bf16  [T, H] in
+ *   x               bf16  [T, H] in (not read when x_perm is NULL)
  *   expert_offsets  int32 [E+1] out: expert e owns rows [off[e], off[e+1])
  *   row_of          int32 [T*k] out: routed row of slot i
  *   src             int32 [T*k] out: slot i of routed row r (inverse of row_of)
  *   w_perm          fp32  [T*k] out: w_perm[row_of[i]] = topk_w[i]
- *   x_perm          bf16  [T*k, H] out: x_perm[row_of[i]] = x[i / k]
+ *   x_perm          bf16  [T*k, H] out: x_perm[row_of[i]] = x[i / k];
+ *                   or NULL: the maps and weights only, for
+ *                   moe_grouped_swiglu_ffn_gather, which reads the rows
+ *                   from x itself
  * Inside an expert, rows are in ascending token order.  Ids outside [0, E)
  * are undefined behaviour. */
 MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids,
@@ -203,6 +206,29 @@ MOE_API moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weigh
                                   const void* x_shared, void* shared_out,
                                   void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The grouped expert FFN with the permute's gather fused into its first
+ * loads ([glm5next] MOE_MODULE token permute and forward_prefill_gemm): the
+ * same result as moe_grouped_swiglu_ffn on x_perm[r] = x[src[r] / k], but
+ * routed row r is read straight from token src[r] / k of x, so x_perm is
+ * never written.  The int4 kernels gather while converting the activations
+ * to fp16 (the conversion pass they run anyway).  The bf16 tensor-core
+ * kernel copies four token rows per TMA gather: correct, but on a B200 its
+ * gate/up launch takes about twice as long as with the contiguous token
+ * boxes of moe_grouped_swiglu_ffn, more than the x_perm copy it saves, so
+ * moe_forward keeps the copy for bf16 experts.
+ * The shared expert runs on x in the same launches when shared_out != NULL.
+ *   x               bf16 [T, H]      src int32 [T*k] (moe_permute's)
+ *   expert_offsets  int32 [E+1]      w_perm fp32 [T*k] or NULL
+ *   y_perm          bf16 [T*k, H] out
+ *   shared_out      bf16 [T, H] out, or NULL (no shared expert)
+ * src must be a permutation of [0, T*k) (moe_permute's output); other
+ * values are undefined behaviour. */
+MOE_API moe_status moe_grouped_swiglu_ffn_gather(const moe_config* cfg, const moe_weights* w,
+                                                 const void* x, int32_t T, const int32_t* src,
+                                                 const int32_t* expert_offsets, const float* w_perm,
+                                                 void* y_perm, void* shared_out,
+                                                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Combine ([glm5next] §One all-reduce: shared output and routed slots are
  * added in one combine kernel):
  *   out[t] = bf16( shared_out[t] + sum_{j<k} c_j * y_perm[row_of[t*k + j]] )
@@ -217,6 +243,9 @@ MOE_API moe_status moe_combine(const moe_config* cfg, const void* y_perm,
 
 /* The whole layer in one call: router -> permute -> grouped FFN (routed +
  * shared) -> combine, enqueued on `stream` with no host synchronisation.
+ * bf16 experts: the permute writes x_perm into the workspace and the FFN
+ * loads contiguous token boxes.  int4 experts: the permute writes the maps
+ * only and the FFN gathers the rows as moe_grouped_swiglu_ffn_gather does.
  *   x    bf16 [T, H];  out bf16 [T, H]
  *   topk_ids_opt int32 [T, k] / topk_w_opt fp32 [T, k]: if non-NULL, the
  *   router's selection is also written there. */

@@ -31,7 +31,8 @@ MOE_INT4_MAX_SWIGLU_LIMIT = 255.0
 
 EXPORTED = (
     "moe_status_string", "moe_config_validate", "moe_workspace_size", "moe_workspace_init",
-    "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_combine", "moe_forward", "moe_forward_ep",
+    "moe_router_topk", "moe_permute", "moe_grouped_swiglu_ffn", "moe_grouped_swiglu_ffn_gather", "moe_combine",
+    "moe_forward", "moe_forward_ep",
     "moe_read_device_error", "moe_permute_no_alloc", "moe_selftest_device_timeout", "moe_selftest_pair_timeout",
 )
 MOE_NO_ALLOC_MAX_ROWS = 131072
@@ -96,6 +97,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_router_topk": (ctypes.c_int, [CFG, W, P, I32, P, P, P, SZ, P]),
         "moe_permute": (ctypes.c_int, [CFG, P, P, P, I32, P, P, P, P, P, P, SZ, P]),
         "moe_grouped_swiglu_ffn": (ctypes.c_int, [CFG, W, P, P, P, I32, P, P, P, P, SZ, P]),
+        "moe_grouped_swiglu_ffn_gather": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, P, P, SZ, P]),
         "moe_combine": (ctypes.c_int, [CFG, P, P, P, P, I32, P, P]),
         "moe_forward": (ctypes.c_int, [CFG, W, P, I32, P, P, P, P, SZ, P]),
         "moe_forward_ep": (ctypes.c_int, [CFG, W, I32, I32, P, I32, P, P, P, P, SZ, P]),
@@ -191,6 +193,13 @@ def moe_grouped_swiglu_ffn(cfg, w, x_perm, expert_offsets, w_perm, T, y_perm, x_
         ctypes.byref(cfg), ctypes.byref(w), _ptr(x_perm), _ptr(expert_offsets), _ptr(w_perm), int(T),
         _ptr(y_perm), _ptr(x_shared), _ptr(shared_out), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)), "moe_grouped_swiglu_ffn")
+
+
+def moe_grouped_swiglu_ffn_gather(cfg, w, x, T, src, expert_offsets, w_perm, y_perm, shared_out, ws, stream=None):
+    _check(load_library().moe_grouped_swiglu_ffn_gather(
+        ctypes.byref(cfg), ctypes.byref(w), _ptr(x), int(T), _ptr(src), _ptr(expert_offsets), _ptr(w_perm),
+        _ptr(y_perm), _ptr(shared_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+        "moe_grouped_swiglu_ffn_gather")
 
 
 def moe_combine(cfg, y_perm, row_of, topk_w, shared_out, T, out, stream=None):

@@ -78,8 +78,11 @@ __host__ __device__ constexpr int tok_box_index(int rows_per_cta) {
 
 struct alignas(64) PairParams {
   CUtensorMap tma_w[2];       // weights: gate/up {K, 8, 2, N/8, G} box {64, 8, 2, 8, 1}; down {K, N, G} box {64, 128, 1}
-  CUtensorMap tma_x[2][kTokBoxes];  // tokens {K, rows} box {64, 128 >> i}: a tile copies only the rows it uses
+  CUtensorMap tma_x[2][kTokBoxes];  // tokens {K, rows} box {64, 128 >> i}: a tile copies only the rows it uses;
+                                    // gathered problem: [0] only, {K, tokens} box {64, 1}
   const int32_t* offsets[2];  // grouped problem: [groups+1]; else nullptr
+  const int32_t* gsrc[2];     // gathered problem: slot of each permuted row (token = slot / gk); else nullptr
+  int32_t gk[2];              // slots per token of a gathered problem
   __nv_bfloat16* out[2];      // [rows, N]
   const float* row_scale[2];  // down: per token row (or nullptr)
   int32_t groups[2];
@@ -161,7 +164,9 @@ __device__ __forceinline__ Tile decode(const PairParams& P, const Ctl& c, int t)
   return ti;
 }
 
-template <Kind KIND>
+// GATHER: some problem of the launch reads its token rows through gsrc
+// (then the whole producer warp copies; otherwise its lane 0 alone).
+template <Kind KIND, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_pair_kernel(const __grid_constant__ PairParams P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -196,7 +201,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 4 && lane == 0) {
     for (int p = 0; p < P.nprob; ++p) {
       tma_prefetch_desc(&P.tma_w[p]);
-      for (int b = 0; b < kTokBoxes; ++b) tma_prefetch_desc(&P.tma_x[p][b]);
+      for (int b = 0; b < (P.gsrc[p] != nullptr ? 1 : kTokBoxes); ++b) tma_prefetch_desc(&P.tma_x[p][b]);
     }
   }
   if (warp == 0) {  // per-problem tile counts; grouped problems: offsets + token-tile prefix
@@ -258,38 +263,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------ TMA producer --
-    if (lane == 0) {
+    // Lane 0 takes the tile ids, waits on the ring and copies the weights
+    // (and a contiguous token box).  For a gathered problem every lane copies
+    // token rows 4 lane .. 4 lane + 3 of the CTA's half with one tile::gather4
+    // per chunk, the hidden rows of the tokens the permutation put there.
+    if (GATHER || lane == 0) {  // lanes 1-31 only help gathers
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
       int q = 0;
       uint32_t qph = 0;
-      int t_next = -2;  // next queue position, once fetched
+      int t_next = -2;  // next queue position, once fetched (lane 0)
       for (;;) {
         // Next tile: the first CTA takes it from the launch's queue and
         // publishes it to both CTAs; tiles go out in order to whichever pair
         // asks first, so pairs that drew cheap (ragged) tiles take more.
-        int t;
-        if (leader) {
-          if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, P.wait_ns)) {
-            fail(35);
-            break;
+        int t = -1;
+        int got = 1;
+        if (lane == 0) {
+          if (leader) {
+            if (!mbar_wait_bounded<true>(&c.tq_empty[q], qph ^ 1u, abort_flag, P.wait_ns)) {
+              fail(35);
+              got = 0;
+            } else {
+              if (t_next == -2) t_next = atomicAdd(P.queue, 1);
+              t = t_next < total_tiles ? t_next : -1;
+              t_next = -2;
+              c.tq[q] = t;
+              st_cluster_u32(map_to_rank(smem_u32(&c.tq[q]), 1), static_cast<uint32_t>(t));
+              mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
+              mbar_arrive(&c.tq_full[q]);
+            }
+          } else {
+            if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, P.wait_ns)) {
+              fail(36);
+              got = 0;
+            } else {
+              t = c.tq[q];
+              mbar_arrive_cluster(leader_bar(&c.tq_empty[q]));
+            }
           }
-          if (t_next == -2) t_next = atomicAdd(P.queue, 1);
-          t = t_next < total_tiles ? t_next : -1;
-          t_next = -2;
-          c.tq[q] = t;
-          st_cluster_u32(map_to_rank(smem_u32(&c.tq[q]), 1), static_cast<uint32_t>(t));
-          mbar_arrive_cluster(map_to_rank(smem_u32(&c.tq_full[q]), 1));
-          mbar_arrive(&c.tq_full[q]);
-        } else {
-          if (!mbar_wait_bounded<true>(&c.tq_full[q], qph, abort_flag, P.wait_ns)) {
-            fail(36);
-            break;
-          }
-          t = c.tq[q];
-          mbar_arrive_cluster(leader_bar(&c.tq_empty[q]));
         }
+        if (GATHER) {
+          got = __shfl_sync(0xffffffffu, got, 0);
+          t = __shfl_sync(0xffffffffu, t, 0);
+        }
+        if (!got) break;
         if (++q == QD) {
           q = 0;
           qph ^= 1u;
@@ -297,36 +316,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (t < 0) break;
         const Tile ti = decode(P, c, t);
         const int p = ti.p;
-        const int xrow = ti.row0 + static_cast<int>(rank) * (ti.nmma / 2);
+        const int half = ti.nmma / 2;  // token rows of this CTA (a multiple of 8)
+        const int xrow = ti.row0 + static_cast<int>(rank) * half;
+        const bool gather = GATHER && P.gsrc[p] != nullptr;
+        const bool my_rows = gather && 4 * lane < half;
+        int g[4] = {0, 0, 0, 0};
+        if (my_rows) {
+          // token of permuted row r = slot src[r] / top_k; rows past the
+          // problem's end (padding up to nmma) read token 0 and are never stored
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = xrow + 4 * lane + j;
+            g[j] = r < P.rows[p] ? __ldg(P.gsrc[p] + r) / P.gk[p] : 0;
+          }
+        }
         // the next id is fetched a few stages before this tile's last copy,
         // so the atomic's round trip overlaps the copies
         const int nkb = P.k_blocks[p];
         const int nstage = (nkb + KCH - 1) / KCH;  // the last stage of an odd count holds one chunk
         const int kpre = nstage > 2 ? nstage - 2 : 0;
-        const int xb = tok_box_index(ti.nmma / 2);
-        const uint32_t b_bytes = static_cast<uint32_t>((TOK / 2) >> xb) * BK * 2;  // this CTA's token copy per chunk
+        const int xb = tok_box_index(half);
+        // this CTA's token bytes per chunk: its rows exactly (gather) or its box
+        const uint32_t b_bytes = static_cast<uint32_t>(gather ? half : (TOK / 2) >> xb) * BK * 2;
         for (int st = 0; st < nstage; ++st) {
-          if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns)) {
-            fail(31);
+          int w_ok = 1;
+          if (lane == 0) {
+            if (!mbar_wait_bounded(&c.empty[stage], phase ^ 1u, abort_flag, P.wait_ns)) {
+              fail(31);
+              w_ok = 0;
+            }
+          }
+          if (GATHER) w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) {
             ok = false;
             break;
           }
           const int nk = min(KCH, nkb - st * KCH);
-          if (leader) mbar_arrive_expect_tx(&c.full[stage], 2u * static_cast<uint32_t>(nk) * (A_BYTES + b_bytes));
+          if (lane == 0 && leader)
+            mbar_arrive_expect_tx(&c.full[stage], 2u * static_cast<uint32_t>(nk) * (A_BYTES + b_bytes));
           const uint32_t bar = leader_bar(&c.full[stage]);
           for (int ch = 0; ch < nk; ++ch) {
             const int kc = (st * KCH + ch) * BK;
-            unsigned char* sa = smem_a + stage * A_STAGE + ch * A_BYTES;  // 1024-byte aligned
-            if (KIND == Kind::GateUp) {
-              const int fb = ti.fidx * 16 + static_cast<int>(rank) * 8;  // first 8-feature block
-              tma_load_5d_pair(sa, &P.tma_w[p], kc, 0, 0, fb, ti.g, bar);
-            } else {
-              const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
-              tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
+            unsigned char* sb = smem_b + stage * B_STAGE + ch * B_BYTES;  // 1024-byte aligned
+            if (lane == 0) {
+              unsigned char* sa = smem_a + stage * A_STAGE + ch * A_BYTES;  // 1024-byte aligned
+              if (KIND == Kind::GateUp) {
+                const int fb = ti.fidx * 16 + static_cast<int>(rank) * 8;  // first 8-feature block
+                tma_load_5d_pair(sa, &P.tma_w[p], kc, 0, 0, fb, ti.g, bar);
+              } else {
+                const int n = ti.fidx * 256 + static_cast<int>(rank) * 128;
+                tma_load_3d_pair(sa, &P.tma_w[p], kc, n, ti.g, bar);
+              }
+              if (!gather) tma_load_2d_pair(sb, &P.tma_x[p][xb], kc, xrow, bar);
             }
-            tma_load_2d_pair(smem_b + stage * B_STAGE + ch * B_BYTES, &P.tma_x[p][xb], kc, xrow, bar);
+            if (my_rows) tma_gather4_pair(sb + lane * 512, &P.tma_x[p][0], kc, g[0], g[1], g[2], g[3], bar);
           }
-          if (leader && st == kpre) t_next = atomicAdd(P.queue, 1);
+          if (lane == 0 && leader && st == kpre) t_next = atomicAdd(P.queue, 1);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -335,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         if (!ok) break;
       }
-      if (leader) {
+      if (lane == 0 && leader) {
         // retire from the queue; the last pair of the launch resets it (every
         // pair has taken its final tile id before it retires)
         __threadfence();
@@ -344,8 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           atomicExch(P.queue, 0);
           atomicExch(P.queue + 1, 0);
         }
-      }
-      if (leader) {  // drain: the last copy of each stage (both CTAs' bytes land here)
+        // drain: the last copy of each stage (both CTAs' bytes land here)
         const int nst = issued < STAGES ? issued : STAGES;
         for (int j = 0; j < nst; ++j) {
           const int i = issued - 1 - j;
@@ -583,9 +627,17 @@ bool encode_x(CUtensorMap (&m)[kTokBoxes], const void* base, int rows, int K) {
   return true;
 }
 
+// Hidden rows of the tokens, [tokens, K], read four rows per copy.
+bool encode_x_rows(CUtensorMap* m, const void* base, int tokens, int K) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(tokens)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {BK, 1};
+  return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // CTA pairs that can be resident at once on the current device (a pair must
 // sit in one GPC, so this can be below half the SM count); 0 if unknown.
-template <Kind KIND>
+template <Kind KIND, bool GATHER>
 int resident_pairs() {
   static int cached[64];
   static bool known[64];
@@ -598,7 +650,7 @@ int resident_pairs() {
     lc.blockDim = dim3(THREADS);
     lc.dynamicSmemBytes = kSmem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, ffn_pair_kernel<KIND>, &lc) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_pair_kernel<KIND, GATHER>, &lc) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
@@ -606,6 +658,18 @@ int resident_pairs() {
     known[dev] = true;
   }
   return cached[dev];
+}
+
+template <Kind KIND, bool GATHER>
+cudaError_t start_pair(const PairParams& P, int num_sms, cudaStream_t stream) {
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<KIND, GATHER>),
+                                   static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  int grid = std::max(2, num_sms / 2 * 2);
+  const int pairs = resident_pairs<KIND, GATHER>();
+  if (pairs > 0) grid = std::min(grid, 2 * pairs);
+  ffn_pair_kernel<KIND, GATHER><<<grid, THREADS, kSmem, stream>>>(P);
+  return cudaGetLastError();
 }
 
 template <Kind KIND>
@@ -622,7 +686,14 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
     return cudaErrorInvalidValue;  // one grouped problem per launch (one offsets table in shared memory)
   for (int i = 0; i < np; ++i) {
     const FfnProblem& f = *probs[i];
-    if (!encode_x(P.tma_x[i], f.a, f.rows, f.K)) return cudaErrorInvalidValue;
+    if (f.gather_src != nullptr) {
+      if (KIND != Kind::GateUp || f.offsets == nullptr || f.gather_k < 1 || f.a_rows < 1) return cudaErrorInvalidValue;
+      if (!encode_x_rows(&P.tma_x[i][0], f.a, f.a_rows, f.K)) return cudaErrorInvalidValue;
+      P.gsrc[i] = f.gather_src;
+      P.gk[i] = f.gather_k;
+    } else if (!encode_x(P.tma_x[i], f.a, f.rows, f.K)) {
+      return cudaErrorInvalidValue;
+    }
     const bool okw = KIND == Kind::GateUp ? encode_w_gu(&P.tma_w[i], f.w, f.groups, f.N, f.K)
                                           : encode_w(&P.tma_w[i], f.w, f.groups, f.N, f.K, 128);
     if (!okw) return cudaErrorInvalidValue;
@@ -641,13 +712,9 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
   P.err = err;
   P.queue = queue;
   P.wait_ns = kTimeoutNs;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<KIND>), static_cast<int>(kSmem));
-  if (e != cudaSuccess) return e;
-  int grid = std::max(2, num_sms / 2 * 2);
-  const int pairs = resident_pairs<KIND>();
-  if (pairs > 0) grid = std::min(grid, 2 * pairs);
-  ffn_pair_kernel<KIND><<<grid, THREADS, kSmem, stream>>>(P);
-  return cudaGetLastError();
+  const bool gather = P.gsrc[0] != nullptr || P.gsrc[1] != nullptr;
+  // (only gate/up problems gather; the down projection reads h in row order)
+  return gather ? start_pair<KIND, KIND == Kind::GateUp>(P, num_sms, stream) : start_pair<KIND, false>(P, num_sms, stream);
 }
 
 }  // namespace
@@ -680,10 +747,10 @@ cudaError_t launch_pair_timeout_selftest(void* scratch, int32_t* err, int32_t* q
   P.queue = queue;
   P.wait_ns = 20000000ull;
   P.test_withhold = 1;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<Kind::GateUp>),
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_pair_kernel<Kind::GateUp, false>),
                                    static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  ffn_pair_kernel<Kind::GateUp><<<2, THREADS, kSmem, stream>>>(P);
+  ffn_pair_kernel<Kind::GateUp, false><<<2, THREADS, kSmem, stream>>>(P);
   return cudaGetLastError();
 }
 

@@ -669,22 +669,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }
 
 // Tokens for the gate/up MMA: fp16, each aligned 8 of K in the order
-// {0, 4, 1, 5, 2, 6, 3, 7}.  One thread per 8 values.
-__global__ void __launch_bounds__(256)
-    int4_tokens_prep_kernel(const __nv_bfloat16* __restrict__ x, long long n8, uint4* __restrict__ out) {
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n8) return;
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + idx);
-  const __half2 p0 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));  // x0, x4
-  const __half2 p1 = __floats2half2_rn(bf16hi(v.x), bf16hi(v.z));  // x1, x5
-  const __half2 p2 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));  // x2, x6
-  const __half2 p3 = __floats2half2_rn(bf16hi(v.y), bf16hi(v.w));  // x3, x7
-  uint4 o;
-  o.x = *reinterpret_cast<const uint32_t*>(&p0);
-  o.y = *reinterpret_cast<const uint32_t*>(&p1);
-  o.z = *reinterpret_cast<const uint32_t*>(&p2);
-  o.w = *reinterpret_cast<const uint32_t*>(&p3);
-  out[idx] = o;
+// {0, 4, 1, 5, 2, 6, 3, 7}.  One block per row, one thread per 8 values.
+// gsrc != NULL: row r is token row gsrc[r] / gk of x (the permutation's
+// gather).
+__global__ void __launch_bounds__(128)
+    int4_tokens_prep_kernel(const __nv_bfloat16* __restrict__ x, int k8, const int32_t* __restrict__ gsrc, int gk,
+                            uint4* __restrict__ out) {
+  const int r = blockIdx.x;
+  const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
+  const uint4* in = reinterpret_cast<const uint4*>(x) + static_cast<size_t>(in_row) * k8;
+  uint4* o = out + static_cast<size_t>(r) * k8;
+  for (int c = threadIdx.x; c < k8; c += blockDim.x) {
+    const uint4 v = __ldg(in + c);
+    const __half2 p0 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));  // x0, x4
+    const __half2 p1 = __floats2half2_rn(bf16hi(v.x), bf16hi(v.z));  // x1, x5
+    const __half2 p2 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));  // x2, x6
+    const __half2 p3 = __floats2half2_rn(bf16hi(v.y), bf16hi(v.w));  // x3, x7
+    uint4 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&p0);
+    w.y = *reinterpret_cast<const uint32_t*>(&p1);
+    w.z = *reinterpret_cast<const uint32_t*>(&p2);
+    w.w = *reinterpret_cast<const uint32_t*>(&p3);
+    o[c] = w;
+  }
 }
 
 bool encode_codes_gu(CUtensorMap* m, const void* q, int groups, int N, int K) {
@@ -814,14 +821,14 @@ cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32
 
 bool int4_prefill_preferred(int rows, int E) { return rows >= 32 * E; }
 
-cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                    const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
-                                    void* y_perm, int32_t* err, int32_t* queues, int num_sms, cudaStream_t stream) {
+cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_rows,
+                                    const int32_t* gather_src, const int32_t* offsets, int rows, void* tokens16,
+                                    void* h16, const float* w_perm, void* y_perm, int32_t* err, int32_t* queues,
+                                    int num_sms, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
   if (rows <= 0) return cudaSuccess;
-  const long long n8 = static_cast<long long>(rows) * (H / 8);
-  int4_tokens_prep_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(x_perm), n8, static_cast<uint4*>(tokens16));
+  int4_tokens_prep_kernel<<<rows, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(x_rows), H / 8, gather_src,
+                                                    cfg.top_k, static_cast<uint4*>(tokens16));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_int4_pair<Kind::GateUp>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, I, H, h16, nullptr,

@@ -93,15 +93,18 @@ moe_status check_router_weights(const moe_weights* w) {
     if ((expr) != cudaSuccess) return MOE_ERR_CUDA;     \
   } while (0)
 
-// The grouped FFN on already-permuted rows (routed) plus, optionally, the
-// shared expert on the raw tokens.  cfg.num_experts is the number of experts
-// this call computes (0 allowed: shared expert only), `offsets` their
-// [E + 1] row offsets (absolute rows of x_perm), and w's routed weights hold
-// exactly those experts; e_total is the router's expert count (the int4 path
-// picks its kernel by the average routed rows per expert, R / e_total).
-moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_perm, const int32_t* offsets,
-                   const float* w_perm, int32_t T, void* y_perm, const void* x_shared, void* shared_out, void* ws,
-                   const WsLayout& L, cudaStream_t stream, int e_total) {
+// The grouped FFN on the permuted rows (routed) plus, optionally, the
+// shared expert on the raw tokens.  The routed rows are x_rows itself
+// (gather_src == NULL: x_perm) or gathered from the tokens x_rows [T, H] by
+// the permutation's slot map (row r = token gather_src[r] / top_k) inside the
+// kernels' own loads.  cfg.num_experts is the number of experts this call
+// computes (0 allowed: shared expert only), `offsets` their [E + 1] row
+// offsets (absolute permuted rows), and w's routed weights hold exactly those
+// experts; e_total is the router's expert count (the int4 path picks its
+// kernel by the average routed rows per expert, R / e_total).
+moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_rows, const int32_t* gather_src,
+                   const int32_t* offsets, const float* w_perm, int32_t T, void* y_perm, const void* x_shared,
+                   void* shared_out, void* ws, const WsLayout& L, cudaStream_t stream, int e_total) {
   const int H = cfg.hidden, I = cfg.expert_inter, Is = cfg.shared_inter, E = cfg.num_experts;
   const int R = T * cfg.top_k;
   const bool routed = E > 0;
@@ -130,7 +133,7 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
     MOE_CUDA_TRY(launch_dense_small_ffn(x_shared, T, H, Is, w.shared_w_gate_up, w.shared_w_down, cfg.swiglu_limit,
                                         at<float>(ws, L.small_part), hs, shared_out, err, sms, stream));
   if (!is_int4(cfg)) {
-    FfnProblem r_gu{x_perm, R, offsets, E, w.w_gate_up, I, H, h, nullptr};
+    FfnProblem r_gu{x_rows, R, offsets, E, w.w_gate_up, I, H, h, nullptr, gather_src, cfg.top_k, T};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
     MOE_CUDA_TRY(launch_gemm_gateup(routed ? &r_gu : nullptr, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, qgu,
                                     sms, stream));
@@ -140,22 +143,39 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_pe
     if (prefill_path) {
       // many tokens per expert: dequantise in shared memory, tensor cores
       if (routed)
-        MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_perm, offsets, R, act16, at<void>(ws, L.h), w_perm, y_perm,
-                                             err, tile_queue(ws, kQueueInt4GateUp), sms, stream));
+        MOE_CUDA_TRY(launch_int4_ffn_prefill(cfg, w, x_rows, gather_src, offsets, R, act16, at<void>(ws, L.h), w_perm,
+                                             y_perm, err, tile_queue(ws, kQueueInt4GateUp), sms, stream));
       if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
     } else {
       // gate/up in fp32 into the h region; the SwiGLU is applied while the
       // down projection's activations are prepared
       float* gu = at<float>(ws, L.h);
       float* gu_s = shared_in_gemv ? at<float>(ws, L.small_part) : nullptr;
-      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_perm, offsets, R, act16, gu, shared_in_gemv ? x_shared : nullptr, T,
-                                       gu_s, stream));
+      MOE_CUDA_TRY(launch_w4a16_gateup(cfg, w, x_rows, gather_src, offsets, R, act16, gu,
+                                       shared_in_gemv ? x_shared : nullptr, T, gu_s, stream));
       if (shared_tc) MOE_CUDA_TRY(launch_gemm_gateup(nullptr, &s_gu, cfg.swiglu_limit, err, qgu, sms, stream));
       MOE_CUDA_TRY(launch_w4a16_down(cfg, w, gu, offsets, R, act16, w_perm, y_perm, gu_s, T, hs, shared_out, stream));
     }
     if (shared_tc) MOE_CUDA_TRY(launch_gemm_down(nullptr, &s_d, err, qd, sms, stream));
   }
   return MOE_OK;
+}
+
+// Where the forward's FFN reads the routed rows.  bf16 experts: the permute
+// copies them into the workspace's x_perm and the tensor-core kernel loads
+// contiguous token boxes (its per-row gather4 form, moe_grouped_swiglu_ffn_gather,
+// takes about twice as long: one TMA copy per four 128-byte rows is
+// latency-bound).  int4 experts: the permute writes the maps only and the
+// activation conversion that every int4 kernel runs first gathers the rows.
+struct Rows {
+  void* x_perm;                 // permute output, or nullptr (maps only)
+  const void* x_rows;           // what run_ffn reads
+  const int32_t* gather_src;    // nullptr, or the slot map of a gathered read
+};
+Rows routed_rows(const moe_config& cfg, void* ws, const WsLayout& L, const void* x, const int32_t* src) {
+  if (is_int4(cfg)) return Rows{nullptr, x, src};
+  void* xp = at<void>(ws, L.x_perm);
+  return Rows{xp, xp, nullptr};
 }
 
 }  // namespace
@@ -199,8 +219,10 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.w_perm = take(R * sizeof(float));
   L.block_base = take(static_cast<size_t>(perm_blocks(static_cast<int>(R))) * E * sizeof(int32_t));
   L.local_rank = take(R * sizeof(int32_t));
-  L.x_perm = take(R * H * 2);
   const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
+  // bf16 experts: the forward gathers the routed rows into x_perm (tiled TMA
+  // copies then feed the tensor cores); int4 experts gather while converting
+  L.x_perm = take(int4 ? 0 : R * H * 2);
   L.h = take(int4 ? R * 2 * I * 4 : R * I * 2);  // int4: fp32 gate/up; bf16: h
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
@@ -289,9 +311,11 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids, const flo
                        size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(moe_config_validate(cfg));
   MOE_TRY(check_tokens(*cfg, T));
-  const void* ptrs[] = {topk_ids, topk_w, x, expert_offsets, row_of, src, w_perm, x_perm};
+  const void* ptrs[] = {topk_ids, topk_w, expert_offsets, row_of, src, w_perm};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  // x_perm == NULL: maps and weights only (x is then not read)
+  if (x_perm != nullptr && (x == nullptr || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
@@ -318,8 +342,30 @@ moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weights* w, c
   MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
   if (T == 0) return MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
-  return run_ffn(*cfg, *w, x_perm, expert_offsets, w_perm, T, y_perm, x_shared, shared_out, ws, L, stream,
+  return run_ffn(*cfg, *w, x_perm, nullptr, expert_offsets, w_perm, T, y_perm, x_shared, shared_out, ws, L, stream,
                  cfg->num_experts);
+}
+
+moe_status moe_grouped_swiglu_ffn_gather(const moe_config* cfg, const moe_weights* w, const void* x, int32_t T,
+                                         const int32_t* src, const int32_t* expert_offsets, const float* w_perm,
+                                         void* y_perm, void* shared_out, void* ws, size_t ws_bytes,
+                                         moe_stream_t stream) {
+  MOE_TRY(moe_config_validate(cfg));
+  MOE_TRY(check_tokens(*cfg, T));
+  MOE_TRY(check_expert_weights(*cfg, w));
+  if (x == nullptr || src == nullptr || expert_offsets == nullptr || y_perm == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(src) || !aligned16(expert_offsets) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (w_perm != nullptr && !aligned16(w_perm)) return MOE_ERR_INVALID_ARG;
+  if (shared_out != nullptr) {
+    if (cfg->shared_inter == 0 || !aligned16(shared_out)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_shared_weights(*cfg, w));
+  }
+  MOE_TRY(check_ws(*cfg, T, ws, ws_bytes));
+  if (T == 0) return MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  return run_ffn(*cfg, *w, x, src, expert_offsets, w_perm, T, y_perm, shared_out != nullptr ? x : nullptr, shared_out,
+                 ws, L, stream, cfg->num_experts);
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
@@ -354,15 +400,16 @@ moe_status moe_forward(const moe_config* cfg, const moe_weights* w, const void* 
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* row_of = at<int32_t>(ws, L.row_of);
   float* w_perm = at<float>(ws, L.w_perm);
-  void* x_perm = at<void>(ws, L.x_perm);
-  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, at<int32_t>(ws, L.src), w_perm, x_perm,
+  int32_t* src = at<int32_t>(ws, L.src);
+  const Rows rows = routed_rows(*cfg, ws, L, x, src);
+  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, src, w_perm, rows.x_perm,
                               at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), perm_ticket(ws),
                               stream));
   void* y_perm = at<void>(ws, L.y_perm);
   const bool shared = cfg->shared_inter > 0;
   void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;
-  MOE_TRY(run_ffn(*cfg, *w, x_perm, offsets, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws, L, stream,
-                  cfg->num_experts));
+  MOE_TRY(run_ffn(*cfg, *w, rows.x_rows, rows.gather_src, offsets, w_perm, T, y_perm, shared ? x : nullptr,
+                  shared_out, ws, L, stream, cfg->num_experts));
   return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out, nullptr, 0, stream));
 }
 
@@ -390,8 +437,9 @@ moe_status moe_forward_ep(const moe_config* cfg, const moe_weights* w, int32_t e
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* row_of = at<int32_t>(ws, L.row_of);
   float* w_perm = at<float>(ws, L.w_perm);
-  void* x_perm = at<void>(ws, L.x_perm);
-  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, at<int32_t>(ws, L.src), w_perm, x_perm,
+  int32_t* src = at<int32_t>(ws, L.src);
+  const Rows rows = routed_rows(*cfg, ws, L, x, src);
+  MOE_CUDA_TRY(launch_permute(*cfg, ids, wts, x, T, offsets, row_of, src, w_perm, rows.x_perm,
                               at<int32_t>(ws, L.block_base), at<int32_t>(ws, L.local_rank), perm_ticket(ws), stream,
                               expert_begin, expert_end));
   void* y_perm = at<void>(ws, L.y_perm);
@@ -399,8 +447,8 @@ moe_status moe_forward_ep(const moe_config* cfg, const moe_weights* w, int32_t e
   void* shared_out = shared ? at<void>(ws, L.shared_out) : nullptr;
   moe_config local = *cfg;
   local.num_experts = El;
-  MOE_TRY(run_ffn(local, *w, x_perm, offsets + expert_begin, w_perm, T, y_perm, shared ? x : nullptr, shared_out, ws,
-                  L, stream, cfg->num_experts));
+  MOE_TRY(run_ffn(local, *w, rows.x_rows, rows.gather_src, offsets + expert_begin, w_perm, T, y_perm,
+                  shared ? x : nullptr, shared_out, ws, L, stream, cfg->num_experts));
   return from_cuda(launch_combine(*cfg, y_perm, row_of, nullptr, shared_out, T, out_partial, offsets + expert_begin,
                                   El, stream));
 }

@@ -232,6 +232,19 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Four rows of a 2-D tensor (row coordinates r0..r3, column c0; the map's
+// box is one row high) into four consecutive box rows at smem_dst, issued by
+// either CTA of a pair; bytes complete on the first CTA's barrier.  The
+// map's swizzle applies by shared-memory address, as for a tiled box.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* m, int32_t c0, int32_t r0,
+                                                 int32_t r1, int32_t r2, int32_t r3, uint32_t bar_leader) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.cta_group::2"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar_leader)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* m, int32_t c0, int32_t c1,
                                                  int32_t c2, uint32_t bar_leader) {
   asm volatile(

@@ -58,7 +58,8 @@ inline int perm_blocks(int R) { return std::max(1, (R + kPermChunk - 1) / kPermC
 // block_base: [perm_blocks(T*k) * E] scratch; local_rank: [T*k] scratch;
 // done: a ticket counter that is zero before the launch and left at zero.
 // Hidden rows are copied into x_perm only for experts in [e0, e1) (e1 < 0:
-// every expert); the maps and weights cover every slot.
+// every expert); the maps and weights cover every slot.  x_perm == nullptr:
+// maps and weights only (x unused).
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
                            int32_t* offsets, int32_t* row_of, int32_t* src, float* w_perm, void* x_perm,
                            int32_t* block_base, int32_t* local_rank, int32_t* done, cudaStream_t stream, int e0 = 0,
@@ -83,6 +84,11 @@ struct FfnProblem {
   int N, K;                      // output columns, reduction length
   void* out;                     // bf16 [rows, N]
   const float* row_scale;        // per-row scale (down only) or nullptr
+  // gate/up of a grouped problem may read its rows straight from the tokens:
+  // row r of the problem is row gather_src[r] / gather_k of `a` ([a_rows, K])
+  const int32_t* gather_src = nullptr;
+  int gather_k = 0;
+  int a_rows = 0;
 };
 // queue: the launch's two tile-queue words in the workspace header (zero).
 cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* shared, float limit, int32_t* err,
@@ -98,9 +104,11 @@ cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared,
 // the down projection's activation prep, and down into shared_out.
 constexpr int kW4a16SharedMaxTokens = 32;
 bool w4a16_shared_fusable(int T, int Is);
-cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
-                                int T, float* gu_shared, cudaStream_t stream);
+// x_rows: the permuted rows [rows, H] (gather_src == NULL), or the tokens
+// [T, H] with row r of the routed problem = token gather_src[r] / top_k.
+cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_rows,
+                                const int32_t* gather_src, const int32_t* offsets, int rows, void* act16, float* gu,
+                                const void* x_shared, int T, float* gu_shared, cudaStream_t stream);
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
                               int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
                               int T, void* h_shared, void* shared_out, cudaStream_t stream);
@@ -110,9 +118,11 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
 // tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16; queues:
 // four tile-queue words in the workspace header (gate/up, then down).
 bool int4_prefill_preferred(int rows, int E);
-cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                    const int32_t* offsets, int rows, void* tokens16, void* h16, const float* w_perm,
-                                    void* y_perm, int32_t* err, int32_t* queues, int num_sms, cudaStream_t stream);
+// x_rows / gather_src as for launch_w4a16_gateup.
+cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_rows,
+                                    const int32_t* gather_src, const int32_t* offsets, int rows, void* tokens16,
+                                    void* h16, const float* w_perm, void* y_perm, int32_t* err, int32_t* queues,
+                                    int num_sms, cudaStream_t stream);
 
 // Shared expert for T <= 32 tokens: split-K tensor-core GEMMs streaming the
 // weights across all SMs, then an ordered sum of the K slices.

@@ -7,7 +7,8 @@
 //      turns the counts into per-(chunk, expert) bases = expert offset +
 //      earlier chunks, and writes the expert offsets;
 //   2. scatter: row = base + rank; row_of / src / w_perm, and the 16-byte
-//      vector gather of the token's hidden row into x_perm.
+//      vector gather of the token's hidden row into x_perm -- or the maps
+//      alone, when the grouped FFN gathers the rows in its own loads.
 // No atomic decides an order (the ticket only picks which block scans), so
 // the result is identical run to run.
 #include "moe_internal.h"
@@ -192,6 +193,20 @@ __global__ void __launch_bounds__(256)
   for (; c < n16; c += 32) d[c] = __ldg(s + c);
 }
 
+// Maps only (the grouped FFN gathers the hidden rows itself): one thread per
+// slot writes its routed row, the inverse map and the weight.
+__global__ void __launch_bounds__(256)
+    perm_maps_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int R, int E,
+                     const int32_t* __restrict__ block_base, const int32_t* __restrict__ local_rank,
+                     int32_t* __restrict__ row_of, int32_t* __restrict__ src, float* __restrict__ w_perm) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R) return;
+  const int row = block_base[static_cast<size_t>(i / kPermChunk) * E + ids[i]] + local_rank[i];
+  row_of[i] = row;
+  src[row] = i;
+  w_perm[row] = topk_w[i];
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const float* topk_w, const void* x, int T,
@@ -208,6 +223,11 @@ cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const floa
                                                     sizeof(int32_t)));
   if (e != cudaSuccess) return e;
   perm_count_rank_kernel<<<nb, kPermWarps * 32, smem, stream>>>(ids, R, E, block_base, local_rank, offsets, done);
+  if (x_perm == nullptr) {
+    perm_maps_kernel<<<(R + 255) / 256, 256, 0, stream>>>(ids, topk_w, R, E, block_base, local_rank, row_of, src,
+                                                         w_perm);
+    return cudaGetLastError();
+  }
   perm_scatter_kernel<<<(R + 7) / 8, 256, 0, stream>>>(ids, topk_w, static_cast<const __nv_bfloat16*>(x), R, k, E,
                                                        H, block_base, local_rank, row_of, src, w_perm,
                                                        static_cast<__nv_bfloat16*>(x_perm), e0,

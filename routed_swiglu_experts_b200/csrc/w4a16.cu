@@ -84,23 +84,31 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
 
 __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-// Activations in MMA slot order.  One thread per 8 consecutive values of a
-// row: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16}.
-__global__ void __launch_bounds__(256)
-    w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, long long n8, uint4* __restrict__ act16) {
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= n8) return;
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(act) + idx);
-  const __half2 a04 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));
-  const __half2 b15 = __floats2half2_rn(bf16hi(v.x) * 0.0625f, bf16hi(v.z) * 0.0625f);
-  const __half2 a26 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));
-  const __half2 b37 = __floats2half2_rn(bf16hi(v.y) * 0.0625f, bf16hi(v.w) * 0.0625f);
-  uint4 o;
-  o.x = *reinterpret_cast<const uint32_t*>(&a04);
-  o.y = *reinterpret_cast<const uint32_t*>(&b15);
-  o.z = *reinterpret_cast<const uint32_t*>(&a26);
-  o.w = *reinterpret_cast<const uint32_t*>(&b37);
-  act16[idx] = o;
+// Activations in MMA slot order.  One block per row, one thread per 8
+// consecutive values: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6,
+// x3/16, x7/16}.  gsrc != NULL: row r of the output is token row
+// gsrc[r] / gk of act (the permutation's gather, done here instead of in a
+// separate copy).
+__global__ void __launch_bounds__(128)
+    w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, int k8, const int32_t* __restrict__ gsrc, int gk,
+                      uint4* __restrict__ act16) {
+  const int r = blockIdx.x;
+  const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
+  const uint4* in = reinterpret_cast<const uint4*>(act) + static_cast<size_t>(in_row) * k8;
+  uint4* out = act16 + static_cast<size_t>(r) * k8;
+  for (int c = threadIdx.x; c < k8; c += blockDim.x) {
+    const uint4 v = __ldg(in + c);
+    const __half2 a04 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));
+    const __half2 b15 = __floats2half2_rn(bf16hi(v.x) * 0.0625f, bf16hi(v.z) * 0.0625f);
+    const __half2 a26 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));
+    const __half2 b37 = __floats2half2_rn(bf16hi(v.y) * 0.0625f, bf16hi(v.w) * 0.0625f);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&a04);
+    o.y = *reinterpret_cast<const uint32_t*>(&b15);
+    o.z = *reinterpret_cast<const uint32_t*>(&a26);
+    o.w = *reinterpret_cast<const uint32_t*>(&b37);
+    out[c] = o;
+  }
 }
 
 // Down-projection activations: the clamped SwiGLU of the fp32 gate/up
@@ -386,10 +394,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
   }
 }
 
-cudaError_t launch_prep(const void* act, int rows, int K, void* act16, cudaStream_t stream) {
-  const long long n8 = static_cast<long long>(rows) * (K / 8);
-  w4a16_prep_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(act), n8, static_cast<uint4*>(act16));
+cudaError_t launch_prep(const void* act, int rows, int K, const int32_t* gsrc, int gk, void* act16,
+                        cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  w4a16_prep_kernel<<<rows, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(act), K / 8, gsrc, gk,
+                                              static_cast<uint4*>(act16));
   return cudaGetLastError();
 }
 
@@ -410,11 +419,11 @@ cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, 
 
 bool w4a16_shared_fusable(int T, int Is) { return Is > 0 && T >= 1 && T <= kW4a16SharedMaxTokens; }
 
-cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_perm,
-                                const int32_t* offsets, int rows, void* act16, float* gu, const void* x_shared,
-                                int T, float* gu_shared, cudaStream_t stream) {
+cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, const void* x_rows,
+                                const int32_t* gather_src, const int32_t* offsets, int rows, void* act16, float* gu,
+                                const void* x_shared, int T, float* gu_shared, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
-  cudaError_t e = launch_prep(x_perm, rows, H, act16, stream);
+  cudaError_t e = launch_prep(x_rows, rows, H, gather_src, cfg.top_k, act16, stream);
   if (e != cudaSuccess) return e;
   SharedJob sj{};
   if (x_shared != nullptr)  // shared gate/up [2 I_s, H] x tokens [T, H] -> fp32 [T, 2 I_s]

@@ -50,10 +50,15 @@ class StageOut:
     y_perm: torch.Tensor
     shared_out: Optional[torch.Tensor]
     out: torch.Tensor
+    # the fused-gather variant: maps-only permute, then the FFN reading x
+    maps: tuple = ()
+    y_perm_g: Optional[torch.Tensor] = None
+    shared_out_g: Optional[torch.Tensor] = None
 
 
 def run_stages(layer: rse.MoELayer, x: torch.Tensor) -> StageOut:
-    """router -> permute -> grouped FFN (+ shared) -> combine, one C-ABI call each."""
+    """router -> permute -> grouped FFN (+ shared) -> combine, one C-ABI call
+    each; then the maps-only permute and the gathered FFN on the same ids."""
     cfg = layer.cfg
     T, H, E, k = x.shape[0], cfg.hidden, cfg.num_experts, cfg.top_k
     R = T * k
@@ -75,8 +80,15 @@ def run_stages(layer: rse.MoELayer, x: torch.Tensor) -> StageOut:
                                x if cfg.shared_inter > 0 else None, shared_out, layer.ws)
     out = torch.empty(T, H, dtype=bf, device=dev)
     rse.moe_combine(cfg, y_perm, row_of, None, shared_out, T, out)
+    maps = tuple(torch.full_like(a, -7) if a.dtype == i32 else torch.full_like(a, -7.0)
+                 for a in (offsets, row_of, src, w_perm))
+    rse.moe_permute(cfg, ids, tw, None, T, *maps, None, layer.ws)
+    y_perm_g = torch.empty(R, H, dtype=bf, device=dev)
+    shared_out_g = torch.empty(T, H, dtype=bf, device=dev) if cfg.shared_inter > 0 else None
+    rse.moe_grouped_swiglu_ffn_gather(cfg, layer.w, x, T, maps[2], maps[0], maps[3], y_perm_g, shared_out_g, layer.ws)
     torch.cuda.synchronize()
-    return StageOut(ids, tw, offsets, row_of, src, w_perm, x_perm, y_perm, shared_out, out)
+    return StageOut(ids, tw, offsets, row_of, src, w_perm, x_perm, y_perm, shared_out, out, maps, y_perm_g,
+                    shared_out_g)
 
 
 def rel_err(got: torch.Tensor, want: torch.Tensor) -> float:

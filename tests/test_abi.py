@@ -98,6 +98,10 @@ def test_workspace_size(lib):
     assert 0 < n0 < n1
     R, H, I = 4096 * 6, 2048, 1408
     assert n1 >= 2 * R * H * 2 + R * I * 2      # x_perm + y_perm + h at least
+    # int4 experts gather their rows while converting them: no x_perm region
+    c4 = mid_cfg(expert_format=_abi.MOE_W_INT4_G128, expert_inter=2048, hidden=2048)
+    R4, I4 = 4096 * 6, 2048
+    assert _abi.moe_workspace_size(c4, 4096) < R4 * H * 2 + R4 * 2 * I4 * 4 + R4 * H * 2 + R4 * max(H, I4) * 2 + (64 << 20)
     with pytest.raises(rse.MoEError):
         _abi.moe_workspace_size(cfg, -1)
 
@@ -158,6 +162,27 @@ def test_stage_argument_checks(lib):
     r = lib.moe_grouped_swiglu_ffn(ctypes.byref(cfg), ctypes.byref(w), FAKE, FAKE, FAKE, 16, FAKE, FAKE, None,
                                    FAKE, ws_bytes, None)
     assert r == _abi.MOE_ERR_INVALID_ARG
+    # permute: x_perm NULL means maps only, and x is then not needed
+    r = lib.moe_permute(ctypes.byref(cfg), FAKE, FAKE, None, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws_bytes, None)
+    assert r == _abi.MOE_OK
+    r = lib.moe_permute(ctypes.byref(cfg), FAKE, FAKE, None, 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+    assert r == _abi.MOE_ERR_INVALID_ARG
+    # gathered FFN: x, src, offsets and y_perm are required; shared_out needs a shared expert
+    def ffn_gather(x=FAKE, T=16, src=FAKE, offs=FAKE, w_perm=FAKE, y=FAKE, sh=FAKE, c=cfg, ww=w, nbytes=ws_bytes):
+        return lib.moe_grouped_swiglu_ffn_gather(ctypes.byref(c), ctypes.byref(ww), x, T, src, offs, w_perm, y, sh,
+                                                 FAKE, nbytes, None)
+    assert ffn_gather(T=0) == _abi.MOE_OK
+    assert ffn_gather(x=None) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(src=None) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(src=FAKE_UNALIGNED) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(offs=None) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(y=None) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(w_perm=FAKE_UNALIGNED) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(c=mid_cfg(shared_inter=0)) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(ww=_fake_weights(shared_w_gate_up=None)) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(ww=_fake_weights(w_gate_up=None)) == _abi.MOE_ERR_INVALID_ARG
+    assert ffn_gather(nbytes=ws_bytes - 1) == _abi.MOE_ERR_WORKSPACE
+    assert ffn_gather(c=mid_cfg(shared_inter=0), sh=None, T=0) == _abi.MOE_OK
     r = lib.moe_combine(ctypes.byref(cfg), FAKE, FAKE, None, None, 16, FAKE_UNALIGNED, None)
     assert r == _abi.MOE_ERR_INVALID_ARG
     r = lib.moe_combine(ctypes.byref(cfg), FAKE, FAKE, None, None, 0, FAKE, None)

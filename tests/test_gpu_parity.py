@@ -148,6 +148,9 @@ def test_stages_match_oracle(small_inputs, name):
     assert torch.equal(st.src.cpu().long(), res.perm.src)
     assert torch.equal(st.w_perm.cpu(), st.topk_w.cpu().reshape(-1)[res.perm.src])
     assert torch.equal(st.x_perm.cpu(), inp.x[res.perm.src // k])
+    # maps-only permute: the same maps and weights
+    for got, want in zip(st.maps, (st.offsets, st.row_of, st.src, st.w_perm)):
+        assert torch.equal(got, want)
 
     tol = tol_for(cfg)
     # routed rows: y_perm[r] = w_perm[r] * FFN_e(x[src[r] / k])
@@ -157,6 +160,10 @@ def test_stages_match_oracle(small_inputs, name):
         assert rel_err(st.shared_out, res.shared) <= tol
     err = rel_err(st.out, res.out)
     assert err <= tol, f"{name}: layer output error {err:.3e} (near-ties {n_tie}, mismatched {n_tie_mis})"
+    # the gather fused into the FFN's loads: the same operands, so the same bits
+    assert torch.equal(st.y_perm_g, st.y_perm)
+    if cfg.I_s > 0:
+        assert torch.equal(st.shared_out_g, st.shared_out)
 
     # the one-call forward gives the same bits as the staged calls
     out2 = layer.forward(x)
