@@ -20,7 +20,9 @@ __device__ __forceinline__ void add8(float (&a)[8], const uint4 v, float c) {
   a[7] = fmaf(c, bf16hi(v.w), a[7]);
 }
 
-// One warp per token: lane j < k reads slot j's routed row and weight once,
+// One warp per token (per column slice of its row when there are too few
+// tokens to fill the GPU: blockIdx.y picks the slice): lane j < k reads slot
+// j's routed row and weight once,
 // the warp shares them with shuffles, then walks the hidden row two 16-byte
 // vectors per lane at a time, so every lane keeps (k + 1) x 2 loads in flight
 // and the index work is paid once per token.  Routed rows outside [lo, hi)
@@ -60,9 +62,13 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
     cs[j] = __shfl_sync(0xffffffffu, my_c, j);
   }
   const int n16 = H / 8;  // 16-byte vectors per row
+  // this warp's columns: slice blockIdx.y of gridDim.y, whole 64-vector steps
+  const int step = 32 * kVecPerLane;
+  const int per = (n16 + step * gridDim.y - 1) / (step * gridDim.y) * step;
+  const int c_end = min(n16, per * static_cast<int>(blockIdx.y + 1));
   const uint4* srow = shared != nullptr ? reinterpret_cast<const uint4*>(shared + static_cast<size_t>(t) * H) : nullptr;
   uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H);
-  for (int c0 = lane; c0 < n16; c0 += 32 * kVecPerLane) {
+  for (int c0 = per * static_cast<int>(blockIdx.y) + lane; c0 < c_end; c0 += step) {
     float a[kVecPerLane][8];
 #pragma unroll
     for (int v = 0; v < kVecPerLane; ++v)
@@ -72,7 +78,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 #pragma unroll
       for (int v = 0; v < kVecPerLane; ++v) {
         const int c = c0 + 32 * v;
-        if (c < n16) add8(a[v], __ldg(srow + c), 1.f);
+        if (c < c_end) add8(a[v], __ldg(srow + c), 1.f);
       }
     }
 #pragma unroll
@@ -82,14 +88,14 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 #pragma unroll
         for (int v = 0; v < kVecPerLane; ++v) {
           const int c = c0 + 32 * v;
-          if (c < n16) add8(a[v], __ldg(yr + c), cs[j]);
+          if (c < c_end) add8(a[v], __ldg(yr + c), cs[j]);
         }
       }
     }
 #pragma unroll
     for (int v = 0; v < kVecPerLane; ++v) {
       const int c = c0 + 32 * v;
-      if (c < n16) {
+      if (c < c_end) {
         uint4 o;
         o.x = pack_bf16x2(a[v][0], a[v][1]);
         o.y = pack_bf16x2(a[v][2], a[v][3]);
@@ -106,7 +112,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int32_t* row_of, const float* topk_w,
                            const void* shared_out, int T, void* out, const int32_t* range, int range_len,
                            cudaStream_t stream) {
-  combine_kernel<<<static_cast<unsigned>((T + kCombineWarps - 1) / kCombineWarps), kCombineWarps * 32, 0, stream>>>(
+  // few tokens: split each row into column slices so that about 2048 warps run
+  const int n16 = cfg.hidden / 8;
+  const int slices = std::max(1, std::min((n16 + 63) / 64, (2048 + T - 1) / std::max(T, 1)));
+  const dim3 grid(static_cast<unsigned>((T + kCombineWarps - 1) / kCombineWarps), static_cast<unsigned>(slices));
+  combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(y_perm), row_of, topk_w, static_cast<const __nv_bfloat16*>(shared_out), T,
       cfg.top_k, cfg.hidden, range, range_len, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();

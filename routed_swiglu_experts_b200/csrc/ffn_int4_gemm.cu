@@ -819,7 +819,7 @@ cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32
   return cudaGetLastError();
 }
 
-bool int4_prefill_preferred(int rows, int E) { return rows >= 32 * E; }
+bool int4_prefill_preferred(int rows, int E) { return rows >= kInt4PrefillRowsPerExpert * E; }
 
 cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_rows,
                                     const int32_t* gather_src, const int32_t* offsets, int rows, void* tokens16,

@@ -223,7 +223,10 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   // bf16 experts: the forward gathers the routed rows into x_perm (tiled TMA
   // copies then feed the tensor cores); int4 experts gather while converting
   L.x_perm = take(int4 ? 0 : R * H * 2);
-  L.h = take(int4 ? R * 2 * I * 4 : R * I * 2);  // int4: fp32 gate/up; bf16: h
+  // bf16 h, or the int4 kernels' h: fp16 [R, I] (grouped GEMM) or fp32 gate/up
+  // [R, 2I] (GEMVs, taken only below kInt4PrefillRowsPerExpert rows per expert)
+  const size_t r_gemv = std::min(R, static_cast<size_t>(kInt4PrefillRowsPerExpert) * E);
+  L.h = take(int4 ? std::max(R * I * 2, r_gemv * 2 * I * 4) : R * I * 2);
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
   L.shared_out = take(T * H * 2);

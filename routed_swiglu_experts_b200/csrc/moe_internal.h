@@ -117,6 +117,8 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
 // fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.
 // tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16; queues:
 // four tile-queue words in the workspace header (gate/up, then down).
+// (at least kInt4PrefillRowsPerExpert routed rows per expert on average)
+constexpr int kInt4PrefillRowsPerExpert = 32;
 bool int4_prefill_preferred(int rows, int E);
 // x_rows / gather_src as for launch_w4a16_gateup.
 cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w, const void* x_rows,
