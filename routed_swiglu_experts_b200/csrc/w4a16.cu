@@ -97,8 +97,6 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
   }
 }
 
-__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-
 // Activations in MMA slot order.  One block per row, one thread per 8
 // consecutive values: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6,
 // x3/16, x7/16}.  gsrc != NULL: row r of the output is token row
@@ -107,6 +105,7 @@ __device__ __forceinline__ float bf16_at(const __nv_bfloat16* p) { return __bflo
 __global__ void __launch_bounds__(128)
     w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, int k8, const int32_t* __restrict__ gsrc, int gk,
                       uint4* __restrict__ act16) {
+  pdl_trigger();
   const int r = blockIdx.x;
   const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
   const uint4* in = reinterpret_cast<const uint4*>(act) + static_cast<size_t>(in_row) * k8;
@@ -143,6 +142,8 @@ __device__ __forceinline__ float swiglu_clamped_f(float g, float u, float L) {
 __global__ void __launch_bounds__(256)
     w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
                              const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs) {
+  pdl_wait();
+  pdl_trigger();
   long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n8) {
     idx -= n8;
@@ -274,9 +275,10 @@ struct SharedJob {
 // also loads its token's 64 activation bytes (lanes past the chunk's last
 // token load that token: their output columns are never stored, and
 // unconditional loads save the per-group zero fill, 3% of the kernel's time)
-// and, every 8 groups, one 16-byte word of 8 scales per row, fetched a batch
-// ahead.  A group's first MMA takes a zero accumulator operand instead of
-// zeroed registers.  The gate/up projection runs as one matrix of 2I
+// and its two rows' bf16 scales, one 2-byte load each (cache-resident; holding
+// a batch of 8 scales per row in registers instead cost 16 registers of the
+// 72 and measured 2% slower).  A group's first MMA takes a zero accumulator
+// operand instead of zeroed registers.  The gate/up projection runs as one matrix of 2I
 // rows with fp32 output (the SwiGLU is applied when the down projection's
 // activations are prepared: pairing each gate row with its up row in one
 // MMA tile to apply it in registers measured 0.5% slower); the down projection writes bf16 scaled by the
@@ -300,6 +302,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
                       const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj) {
   extern __shared__ uint4 gemv_ring[];
   constexpr int S = kGemvStages;
+  pdl_wait();  // the activations come from the previous launch
+  pdl_trigger();
   // blocks of the first grid row take the shared expert (when there is one):
   // they start first, and their weight stream runs beside the routed blocks'
   int e = blockIdx.y;
@@ -319,7 +323,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
   if (n0 >= N) return;
   const int groups = K / 128;
   const size_t rb = static_cast<size_t>(K) / 2;
-  const bool batch8 = (groups & 7) == 0;  // scale rows 16-byte aligned every 8 groups
   const size_t row0 = static_cast<size_t>(e) * N + n0 + g;
   const uint8_t* q0 = q + row0 * rb + 16 * t;  // row g; row g + 8 at + q8off
   const uint32_t q8off = 8u * static_cast<uint32_t>(rb);  // < 2^32: a bf16 row of K is < 2^31 bytes
@@ -342,26 +345,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
       cp_async_commit();
     }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    uint4 sv0 = make_uint4(0, 0, 0, 0), sv8 = sv0, sn0 = sv0, sn8 = sv0;
-    if (batch8) {
-      sv0 = __ldg(reinterpret_cast<const uint4*>(s0p));
-      sv8 = __ldg(reinterpret_cast<const uint4*>(s8p));
-      if (groups > 8) {
-        sn0 = __ldg(reinterpret_cast<const uint4*>(s0p + 8));
-        sn8 = __ldg(reinterpret_cast<const uint4*>(s8p + 8));
-      }
-    }
+
     const uint8_t* qb = q0;  // codes of group g0
     const uint4* ab = ap;    // activations of group g0
     for (int g0 = 0; g0 < groups; g0 += 8, qb += 8 * 64, ab += 8 * 16) {
-      if (batch8 && g0 > 0) {
-        sv0 = sn0;
-        sv8 = sn8;
-        if (g0 + 8 < groups) {
-          sn0 = __ldg(reinterpret_cast<const uint4*>(s0p + g0 + 8));
-          sn8 = __ldg(reinterpret_cast<const uint4*>(s8p + g0 + 8));
-        }
-      }
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const int gq = g0 + jj;
@@ -376,16 +363,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
           const uint4 c0 = st[0], c8 = st[32];
           float tt[4];
           tile_group(tt, c0, c8, act);
-          float a0, a8;
-          if (batch8) {
-            const uint32_t w0 = (jj >> 1) == 0 ? sv0.x : (jj >> 1) == 1 ? sv0.y : (jj >> 1) == 2 ? sv0.z : sv0.w;
-            const uint32_t w8 = (jj >> 1) == 0 ? sv8.x : (jj >> 1) == 1 ? sv8.y : (jj >> 1) == 2 ? sv8.z : sv8.w;
-            a0 = (jj & 1) ? bf16hi(w0) : bf16lo(w0);
-            a8 = (jj & 1) ? bf16hi(w8) : bf16lo(w8);
-          } else {
-            a0 = bf16_at(s0p + gq);
-            a8 = bf16_at(s8p + gq);
-          }
+          const float a0 = __bfloat162float(__ldg(s0p + gq)), a8 = __bfloat162float(__ldg(s8p + gq));
           acc[0] = fmaf(a0, tt[0], acc[0]);
           acc[1] = fmaf(a0, tt[1], acc[1]);
           acc[2] = fmaf(a8, tt[2], acc[2]);
@@ -427,10 +405,9 @@ cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, 
   const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
   const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
   if (grid.y == 0) return cudaSuccess;  // no routed expert and no shared expert in this call
-  w4a16_gemv_kernel<F32OUT><<<grid, kGemvWarps * 32, kGemvSmem, stream>>>(
-      static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
-      static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
-  return cudaGetLastError();
+  return launch_after_previous(w4a16_gemv_kernel<F32OUT>, grid, dim3(kGemvWarps * 32), kGemvSmem, stream,
+                               static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
+                               static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
 }
 
 }  // namespace
@@ -458,10 +435,10 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
   const long long n8 = static_cast<long long>(rows) * (I / 8);
   const long long n8s = gu_shared != nullptr ? static_cast<long long>(T) * (Is / 8) : 0;
   if (n8 + n8s > 0) {
-    w4a16_prep_swiglu_kernel<<<static_cast<unsigned>((n8 + n8s + 255) / 256), 256, 0, stream>>>(
-        gu, I, n8, cfg.swiglu_limit, static_cast<uint4*>(act16), gu_shared, Is, n8s,
-        static_cast<__nv_bfloat16*>(h_shared));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_after_previous(w4a16_prep_swiglu_kernel, dim3(static_cast<unsigned>((n8 + n8s + 255) / 256)),
+                                          dim3(256), 0, stream, gu, I, n8, cfg.swiglu_limit,
+                                          static_cast<uint4*>(act16), gu_shared, Is, n8s,
+                                          static_cast<__nv_bfloat16*>(h_shared));
     if (e != cudaSuccess) return e;
   }
   SharedJob sj{};
