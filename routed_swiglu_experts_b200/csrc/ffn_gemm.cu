@@ -169,6 +169,8 @@ __device__ __forceinline__ Tile decode(const PairParams& P, const Ctl& c, int t)
 template <Kind KIND, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_pair_kernel(const __grid_constant__ PairParams P) {
+  pdl_wait();  // the previous launch on the stream has finished
+  pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -668,8 +670,7 @@ cudaError_t start_pair(const PairParams& P, int num_sms, cudaStream_t stream) {
   int grid = std::max(2, num_sms / 2 * 2);
   const int pairs = resident_pairs<KIND, GATHER>();
   if (pairs > 0) grid = std::min(grid, 2 * pairs);
-  ffn_pair_kernel<KIND, GATHER><<<grid, THREADS, kSmem, stream>>>(P);
-  return cudaGetLastError();
+  return launch_after_previous(ffn_pair_kernel<KIND, GATHER>, dim3(grid), dim3(THREADS), kSmem, stream, P);
 }
 
 template <Kind KIND>

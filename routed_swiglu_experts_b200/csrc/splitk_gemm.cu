@@ -113,6 +113,8 @@ __device__ __forceinline__ void tile_k_range(const SplitKParams& P, const TileIn
 }
 
 __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_constant__ SplitKParams P) {
+  pdl_wait();  // the previous launch on the stream has finished
+  pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -398,8 +400,8 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemMax));
   if (e != cudaSuccess) return e;
   const int tiles = ((rows + BM - 1) / BM) * P.n_tiles;
-  splitk_gemm_kernel<<<std::min(num_sms, tiles), THREADS, smem_bytes(P), stream>>>(P);
-  return cudaGetLastError();
+  return launch_after_previous(splitk_gemm_kernel, dim3(std::min(num_sms, tiles)), dim3(THREADS), smem_bytes(P),
+                               stream, P);
 }
 
 // Test hook: one 128 x 16 x 64 tile over zero operands in `scratch` whose

@@ -105,6 +105,7 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
 __global__ void __launch_bounds__(128)
     w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, int k8, const int32_t* __restrict__ gsrc, int gk,
                       uint4* __restrict__ act16) {
+  pdl_wait();  // the previous launch on the stream has finished
   pdl_trigger();
   const int r = blockIdx.x;
   const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
@@ -393,9 +394,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
 cudaError_t launch_prep(const void* act, int rows, int K, const int32_t* gsrc, int gk, void* act16,
                         cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  w4a16_prep_kernel<<<rows, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(act), K / 8, gsrc, gk,
-                                              static_cast<uint4*>(act16));
-  return cudaGetLastError();
+  return launch_after_previous(w4a16_prep_kernel, dim3(rows), dim3(128), 0, stream,
+                               static_cast<const __nv_bfloat16*>(act), K / 8, gsrc, gk, static_cast<uint4*>(act16));
 }
 
 template <bool F32OUT>
