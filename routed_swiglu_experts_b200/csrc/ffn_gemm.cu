@@ -169,7 +169,6 @@ __device__ __forceinline__ Tile decode(const PairParams& P, const Ctl& c, int t)
 template <Kind KIND, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_pair_kernel(const __grid_constant__ PairParams P) {
-  pdl_wait();  // the previous launch on the stream has finished
   pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -206,6 +205,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int b = 0; b < (P.gsrc[p] != nullptr ? 1 : kTokBoxes); ++b) tma_prefetch_desc(&P.tma_x[p][b]);
     }
   }
+  // TMEM and the tensor maps are this launch's own: taken before waiting for
+  // the previous launch on the stream, so that their latency overlaps its tail
+  if (warp == 5) tmem_alloc_pair(&c.tmem_base, TMEM_COLS);
+  pdl_wait();  // every global access below comes after the previous launch has finished
   if (warp == 0) {  // per-problem tile counts; grouped problems: offsets + token-tile prefix
     for (int p = 0; p < 2; ++p) {
       int tiles = 0;
@@ -249,7 +252,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (lane == 0) c.tiles[p] = tiles;
     }
   }
-  if (warp == 5) tmem_alloc_pair(&c.tmem_base, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive

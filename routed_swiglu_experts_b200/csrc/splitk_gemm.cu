@@ -113,7 +113,6 @@ __device__ __forceinline__ void tile_k_range(const SplitKParams& P, const TileIn
 }
 
 __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_constant__ SplitKParams P) {
-  pdl_wait();  // the previous launch on the stream has finished
   pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -142,6 +141,9 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
     tma_prefetch_desc(&P.tma_b);
   }
   if (warp == 5) tmem_alloc(&c.tmem_base, TMEM_COLS);
+  // barriers, TMEM and the tensor-map prefetch overlap the previous launch's
+  // tail; every global access comes after it has finished
+  pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
