@@ -8,8 +8,10 @@ output, the shared-expert output and every routed row of the compared
 tokens: all tokens of the mid and decode layers, and on the larger layers a
 sample of at least 1024 tokens chosen per token tile (the first and last
 rows of every tile of every expert, and the rows where a tile's two CTA
-halves meet).  Near-tie counts go into every assertion message and the
-test's printed line.
+halves meet).  The maps-only permute and the grouped FFN with the gather
+fused into its loads are compared bit for bit with the x_perm path on every
+layer.  Near-tie counts go into every assertion message and the test's
+printed line.
 
 Bars: expert ids and permutation indices bit-exact (router ids exempt only
 where the oracle's k-th vs (k+1)-th biased-score gap is below 1e-6; those
@@ -298,6 +300,13 @@ def test_full_size_layer(name):
     # permutation for every slot
     perm = oracle.permute(gpu_ids, cfg.E)
     assert torch.equal(st.offsets.cpu().long(), perm.expert_offsets), ties
+    # the maps-only permute and the FFN with the gather fused into its loads
+    # give the x_perm path's maps and bits at full size as well
+    for got, want in zip(st.maps, (st.offsets, st.row_of, st.src, st.w_perm)):
+        assert torch.equal(got, want)
+    assert torch.equal(st.y_perm_g, st.y_perm)
+    if cfg.I_s > 0:
+        assert torch.equal(st.shared_out_g, st.shared_out)
     assert torch.equal(st.row_of.cpu().long(), perm.row_of), ties
     assert torch.equal(st.src.cpu().long(), perm.src), ties
     src_dev = st.src.long()
