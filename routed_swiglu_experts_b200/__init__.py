@@ -17,7 +17,8 @@ from ._abi import (  # noqa: F401
     EXPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
     MOE_ERR_WORKSPACE, MOE_MAX_EXPERTS, MOE_MAX_TOP_K, MOE_OK, MOE_W_BF16, MOE_W_INT4_G128, MoEError,
     load_library, make_config, make_weights, moe_combine, moe_config, moe_config_validate, moe_forward,
-    moe_grouped_swiglu_ffn, moe_grouped_swiglu_ffn_gather, moe_permute, moe_read_device_error, moe_router_topk, moe_weights,
+    moe_grouped_swiglu_ffn, moe_grouped_swiglu_ffn_gather, moe_permute, moe_read_device_error, moe_router_topk,
+    moe_weights,
     moe_workspace_init, moe_workspace_size, status_name,
 )
 

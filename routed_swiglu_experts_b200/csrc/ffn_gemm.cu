@@ -717,7 +717,8 @@ cudaError_t launch_pair(const FfnProblem* routed, const FfnProblem* shared, floa
   P.wait_ns = kTimeoutNs;
   const bool gather = P.gsrc[0] != nullptr || P.gsrc[1] != nullptr;
   // (only gate/up problems gather; the down projection reads h in row order)
-  return gather ? start_pair<KIND, KIND == Kind::GateUp>(P, num_sms, stream) : start_pair<KIND, false>(P, num_sms, stream);
+  return gather ? start_pair<KIND, KIND == Kind::GateUp>(P, num_sms, stream)
+                : start_pair<KIND, false>(P, num_sms, stream);
 }
 
 }  // namespace
