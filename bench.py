@@ -314,7 +314,11 @@ def measure_decode(dev, iters, clocks, max_over_ranks):
     beside the mid layer's line: its expert FFN call (the HBM-bound part:
     codes and scales of every touched expert, the bf16 shared expert) and
     its whole forward, each timed with CUDA events over `iters` calls after
-    warm-up.  The touched experts' codes alone (about 2.9 GB) exceed L2."""
+    warm-up, a burst of at most 50 (the HBM peak it is compared with is a
+    copy timed on its own; the call is bound by its instruction stream, so
+    a longer loop measures how far the power cap pulls the clock down).  The
+    touched experts' codes alone (about 2.9 GB) exceed L2, so every call
+    streams them from HBM."""
     import torch
     import routed_swiglu_experts_b200 as rse
     cfg, inp = make_inputs(DECODE_NAME)
@@ -545,7 +549,7 @@ def bench_ours(args, rank, world, local_rank):
         # own, so it is timed after the host-side oracle baseline (about 10 s
         # with the GPU idle), not in the clock state the mid layer's long runs
         # leave behind under the power cap
-        decode = measure_decode(dev, max(20, min(args.steps, 200)), clocks, max_over_ranks)
+        decode = measure_decode(dev, max(20, min(args.steps, 50)), clocks, max_over_ranks)
     clk = clocks.finish()
 
     peaks = measured_peaks()
