@@ -36,8 +36,6 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const __nv_bfloat16* __restrict__ y_perm, const int32_t* __restrict__ row_of,
                    const float* __restrict__ topk_w, const __nv_bfloat16* __restrict__ shared, int T, int k, int H,
                    const int32_t* __restrict__ range, int range_len, __nv_bfloat16* __restrict__ out) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= T) return;
@@ -120,7 +118,7 @@ cudaError_t launch_combine(const moe_config& cfg, const void* y_perm, const int3
   constexpr int step = 32 * kVecPerLane;  // 16-byte vectors a warp covers per pass
   const int slices = std::max(1, std::min((n16 + step - 1) / step, (2048 + T - 1) / std::max(T, 1)));
   const dim3 grid(static_cast<unsigned>((T + kCombineWarps - 1) / kCombineWarps), static_cast<unsigned>(slices));
-  return launch_after_previous(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream,
+  return launch_kernel(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream,
                                static_cast<const __nv_bfloat16*>(y_perm), row_of, topk_w,
                                static_cast<const __nv_bfloat16*>(shared_out), T, cfg.top_k, cfg.hidden, range,
                                range_len, static_cast<__nv_bfloat16*>(out));

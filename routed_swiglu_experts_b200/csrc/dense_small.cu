@@ -23,8 +23,6 @@ constexpr int kMmaN = 256;
 __global__ void __launch_bounds__(256)
     dense_small_finish_kernel(const float* __restrict__ part, int S, int T, int ncols, int gate_up, int cols,
                               float L, __nv_bfloat16* __restrict__ out) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int c4 = cols / 4;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // over T * cols / 4
   if (idx >= T * c4) return;
@@ -81,14 +79,14 @@ cudaError_t launch_dense_small_ffn(const void* x, int T, int H, int Is, const vo
   int S = splits_for(2 * Is, H, T, num_sms);
   cudaError_t e = launch_splitk_gemm(x, T, H, w_gu, 1, 2 * Is, kMmaN, S, part, err, num_sms, stream);
   if (e != cudaSuccess) return e;
-  e = launch_after_previous(dense_small_finish_kernel, dim3((T * Is / 4 + 255) / 256), dim3(256), 0, stream,
+  e = launch_kernel(dense_small_finish_kernel, dim3((T * Is / 4 + 255) / 256), dim3(256), 0, stream,
                             static_cast<const float*>(part), S, T, 2 * Is, 1, Is, L, static_cast<__nv_bfloat16*>(h_s));
   if (e != cudaSuccess) return e;
   // down: [T, I_s] x [H, I_s]^T
   S = splits_for(H, Is, T, num_sms);
   e = launch_splitk_gemm(h_s, T, Is, w_d, 1, H, kMmaN, S, part, err, num_sms, stream);
   if (e != cudaSuccess) return e;
-  return launch_after_previous(dense_small_finish_kernel, dim3((T * H / 4 + 255) / 256), dim3(256), 0, stream,
+  return launch_kernel(dense_small_finish_kernel, dim3((T * H / 4 + 255) / 256), dim3(256), 0, stream,
                                static_cast<const float*>(part), S, T, H, 0, H, 0.f, static_cast<__nv_bfloat16*>(out));
 }
 

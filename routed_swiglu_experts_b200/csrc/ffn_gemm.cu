@@ -169,7 +169,6 @@ __device__ __forceinline__ Tile decode(const PairParams& P, const Ctl& c, int t)
 template <Kind KIND, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_pair_kernel(const __grid_constant__ PairParams P) {
-  pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -205,10 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       for (int b = 0; b < (P.gsrc[p] != nullptr ? 1 : kTokBoxes); ++b) tma_prefetch_desc(&P.tma_x[p][b]);
     }
   }
-  // TMEM and the tensor maps are this launch's own: taken before waiting for
-  // the previous launch on the stream, so that their latency overlaps its tail
   if (warp == 5) tmem_alloc_pair(&c.tmem_base, TMEM_COLS);
-  pdl_wait();  // every global access below comes after the previous launch has finished
   if (warp == 0) {  // per-problem tile counts; grouped problems: offsets + token-tile prefix
     for (int p = 0; p < 2; ++p) {
       int tiles = 0;
@@ -672,7 +668,7 @@ cudaError_t start_pair(const PairParams& P, int num_sms, cudaStream_t stream) {
   int grid = std::max(2, num_sms / 2 * 2);
   const int pairs = resident_pairs<KIND, GATHER>();
   if (pairs > 0) grid = std::min(grid, 2 * pairs);
-  return launch_after_previous(ffn_pair_kernel<KIND, GATHER>, dim3(grid), dim3(THREADS), kSmem, stream, P);
+  return launch_kernel(ffn_pair_kernel<KIND, GATHER>, dim3(grid), dim3(THREADS), kSmem, stream, P);
 }
 
 template <Kind KIND>

@@ -179,8 +179,6 @@ __device__ __forceinline__ int slot_of(int f) {
 template <Kind KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_int4_pair_kernel(const __grid_constant__ Int4Params P) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -677,8 +675,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 __global__ void __launch_bounds__(128)
     int4_tokens_prep_kernel(const __nv_bfloat16* __restrict__ x, int k8, const int32_t* __restrict__ gsrc, int gk,
                             uint4* __restrict__ out) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int r = blockIdx.x;
   const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
   const uint4* in = reinterpret_cast<const uint4*>(x) + static_cast<size_t>(in_row) * k8;
@@ -776,7 +772,7 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
   int grid = std::max(2, num_sms / 2 * 2);
   const int pairs = resident_pairs_int4<KIND>();
   if (pairs > 0) grid = std::min(grid, 2 * pairs);
-  return launch_after_previous(ffn_int4_pair_kernel<KIND>, dim3(grid), dim3(THREADS), kSmem, stream, P);
+  return launch_kernel(ffn_int4_pair_kernel<KIND>, dim3(grid), dim3(THREADS), kSmem, stream, P);
 }
 
 }  // namespace
@@ -830,7 +826,7 @@ cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w,
                                     int num_sms, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
   if (rows <= 0) return cudaSuccess;
-  cudaError_t e = launch_after_previous(int4_tokens_prep_kernel, dim3(rows), dim3(128), 0, stream,
+  cudaError_t e = launch_kernel(int4_tokens_prep_kernel, dim3(rows), dim3(128), 0, stream,
                                         static_cast<const __nv_bfloat16*>(x_rows), H / 8, gather_src, cfg.top_k,
                                         static_cast<uint4*>(tokens16));
   if (e != cudaSuccess) return e;

@@ -111,16 +111,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
-// ------------------------------------------- programmatic dependent launch --
-// A kernel launched with programmatic stream serialization may start before
-// the previous kernel on its stream has finished; pdl_wait() blocks until that
-// kernel has completed and its memory is visible (a no-op for an ordinary
-// launch), so it comes before the kernel's first global access.
-// pdl_trigger() lets the next such kernel be scheduled once every block of
-// this one has issued it.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // ------------------------------------------------------------- cp.async ---
 // 16-byte global -> shared copy that bypasses L1; visible to the issuing
 // thread after cp_async_wait.

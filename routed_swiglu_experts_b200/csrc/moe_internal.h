@@ -14,22 +14,16 @@ namespace moe {
 // (cached per device and kernel).
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 
-// Launch `kernel` with programmatic stream serialization: it may be
-// scheduled while the previous kernel on `stream` is finishing, and must call
-// pdl_wait() before its first global memory access.
+// Launch `kernel` on `stream` (an ordinary, fully ordered launch) and
+// return the launch status.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_after_previous(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                                  Args&&... args) {
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args&&... args) {
   cudaLaunchConfig_t lc = {};
   lc.gridDim = grid;
   lc.blockDim = block;
   lc.dynamicSmemBytes = smem;
   lc.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
   return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
 }
 

@@ -50,8 +50,6 @@ __global__ void __launch_bounds__(kPermWarps * 32)
     perm_count_rank_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* __restrict__ block_base,
                            int32_t* __restrict__ local_rank, int32_t* __restrict__ offsets,
                            int32_t* __restrict__ done) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   extern __shared__ int32_t cnt[];
   __shared__ int32_t tot[MOE_MAX_EXPERTS];
   __shared__ int32_t wsum[kPermWarps];
@@ -170,8 +168,6 @@ __global__ void __launch_bounds__(256)
                         const int32_t* __restrict__ block_base, const int32_t* __restrict__ local_rank,
                         int32_t* __restrict__ row_of, int32_t* __restrict__ src, float* __restrict__ w_perm,
                         __nv_bfloat16* __restrict__ x_perm, int e0, int e1) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (i >= R) return;
@@ -203,8 +199,6 @@ __global__ void __launch_bounds__(256)
     perm_maps_kernel(const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int R, int E,
                      const int32_t* __restrict__ block_base, const int32_t* __restrict__ local_rank,
                      int32_t* __restrict__ row_of, int32_t* __restrict__ src, float* __restrict__ w_perm) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= R) return;
   const int row = block_base[static_cast<size_t>(i / kPermChunk) * E + ids[i]] + local_rank[i];
@@ -228,14 +222,14 @@ cudaError_t launch_permute(const moe_config& cfg, const int32_t* ids, const floa
                                    static_cast<int>(std::max(kPermWarps * MOE_MAX_EXPERTS, kScanSmemEntries) *
                                                     sizeof(int32_t)));
   if (e != cudaSuccess) return e;
-  e = launch_after_previous(perm_count_rank_kernel, dim3(nb), dim3(kPermWarps * 32), smem, stream, ids, R, E,
+  e = launch_kernel(perm_count_rank_kernel, dim3(nb), dim3(kPermWarps * 32), smem, stream, ids, R, E,
                             block_base, local_rank, offsets, done);
   if (e != cudaSuccess) return e;
   if (x_perm == nullptr)
-    return launch_after_previous(perm_maps_kernel, dim3((R + 255) / 256), dim3(256), 0, stream, ids, topk_w, R, E,
+    return launch_kernel(perm_maps_kernel, dim3((R + 255) / 256), dim3(256), 0, stream, ids, topk_w, R, E,
                                  static_cast<const int32_t*>(block_base), static_cast<const int32_t*>(local_rank),
                                  row_of, src, w_perm);
-  return launch_after_previous(perm_scatter_kernel, dim3((R + 7) / 8), dim3(256), 0, stream, ids, topk_w,
+  return launch_kernel(perm_scatter_kernel, dim3((R + 7) / 8), dim3(256), 0, stream, ids, topk_w,
                                static_cast<const __nv_bfloat16*>(x), R, k, E, H,
                                static_cast<const int32_t*>(block_base), static_cast<const int32_t*>(local_rank),
                                row_of, src, w_perm, static_cast<__nv_bfloat16*>(x_perm), e0, e1 < 0 ? E : e1);

@@ -20,8 +20,6 @@ namespace {
 // of w itself.  Output [3, E, H] (part-major) for the tensor-core GEMM.
 __global__ void __launch_bounds__(256)
     router_split_kernel(const float4* __restrict__ wr, int n4, uint2* __restrict__ parts) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   const float4 w = __ldg(wr + i);
@@ -286,8 +284,6 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
                             const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H, int k,
                             float alpha, int renorm, float tau, int32_t* __restrict__ ids_out,
                             float* __restrict__ w_out) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int s_n;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -362,8 +358,6 @@ __global__ void __launch_bounds__(kRowsThreads)
                             const float* __restrict__ wr, const float* __restrict__ bias, int T, int E, int H, int k,
                             float alpha, int renorm, float tau, int tb, int32_t* __restrict__ ids_out,
                             float* __restrict__ w_out) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const size_t pw = rows_scratch_per_warp(E);
@@ -475,7 +469,7 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
   const int E = cfg.num_experts, H = cfg.hidden, k = cfg.top_k;
   const RouterPlan p = router_plan(T, E, H, num_sms);
   const int n4 = E * H / 4;
-  cudaError_t err_c = launch_after_previous(router_split_kernel, dim3((n4 + 255) / 256), dim3(256), 0, stream,
+  cudaError_t err_c = launch_kernel(router_split_kernel, dim3((n4 + 255) / 256), dim3(256), 0, stream,
                                             reinterpret_cast<const float4*>(w.router_w), n4,
                                             static_cast<uint2*>(w_split));
   if (err_c != cudaSuccess) return err_c;
@@ -487,7 +481,7 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
     err_c = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_coop_kernel),
                              static_cast<int>(router_topk_smem(MOE_MAX_EXPERTS)));
     if (err_c != cudaSuccess) return err_c;
-    return launch_after_previous(router_topk_coop_kernel, dim3(T), dim3(kTopkWarps * 32), router_topk_smem(E),
+    return launch_kernel(router_topk_coop_kernel, dim3(T), dim3(kTopkWarps * 32), router_topk_smem(E),
                                  stream, static_cast<const float*>(part), p.ks, xb, w.router_w, w.correction_bias, T,
                                  E, H, k, cfg.routed_scaling_factor, cfg.renormalize, kRouterTieTau, ids, wts);
   }
@@ -495,7 +489,7 @@ cudaError_t launch_router(const moe_config& cfg, const moe_weights& w, const voi
   err_c = ensure_smem_attr(reinterpret_cast<const void*>(router_topk_rows_kernel),
                            static_cast<int>(rows_smem(MOE_MAX_EXPERTS, rows_tokens_per_block(MOE_MAX_EXPERTS))));
   if (err_c != cudaSuccess) return err_c;
-  return launch_after_previous(router_topk_rows_kernel, dim3(static_cast<unsigned>((T + tb - 1) / tb)),
+  return launch_kernel(router_topk_rows_kernel, dim3(static_cast<unsigned>((T + tb - 1) / tb)),
                                dim3(kRowsThreads), rows_smem(E, tb), stream, static_cast<const float*>(part), p.ks,
                                xb, w.router_w, w.correction_bias, T, E, H, k, cfg.routed_scaling_factor,
                                cfg.renormalize, kRouterTieTau, tb, ids, wts);

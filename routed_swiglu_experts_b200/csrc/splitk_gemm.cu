@@ -113,7 +113,6 @@ __device__ __forceinline__ void tile_k_range(const SplitKParams& P, const TileIn
 }
 
 __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_constant__ SplitKParams P) {
-  pdl_trigger();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -141,9 +140,6 @@ __global__ void __launch_bounds__(THREADS, 1) splitk_gemm_kernel(const __grid_co
     tma_prefetch_desc(&P.tma_b);
   }
   if (warp == 5) tmem_alloc(&c.tmem_base, TMEM_COLS);
-  // barriers, TMEM and the tensor-map prefetch overlap the previous launch's
-  // tail; every global access comes after it has finished
-  pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -402,7 +398,7 @@ cudaError_t launch_splitk_gemm(const void* a, int rows, int K, const void* b, in
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(splitk_gemm_kernel), static_cast<int>(kSmemMax));
   if (e != cudaSuccess) return e;
   const int tiles = ((rows + BM - 1) / BM) * P.n_tiles;
-  return launch_after_previous(splitk_gemm_kernel, dim3(std::min(num_sms, tiles)), dim3(THREADS), smem_bytes(P),
+  return launch_kernel(splitk_gemm_kernel, dim3(std::min(num_sms, tiles)), dim3(THREADS), smem_bytes(P),
                                stream, P);
 }
 

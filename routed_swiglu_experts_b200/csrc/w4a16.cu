@@ -105,8 +105,6 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
 __global__ void __launch_bounds__(128)
     w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, int k8, const int32_t* __restrict__ gsrc, int gk,
                       uint4* __restrict__ act16) {
-  pdl_wait();  // the previous launch on the stream has finished
-  pdl_trigger();
   const int r = blockIdx.x;
   const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
   const uint4* in = reinterpret_cast<const uint4*>(act) + static_cast<size_t>(in_row) * k8;
@@ -143,8 +141,6 @@ __device__ __forceinline__ float swiglu_clamped_f(float g, float u, float L) {
 __global__ void __launch_bounds__(256)
     w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
                              const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs) {
-  pdl_wait();
-  pdl_trigger();
   long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n8) {
     idx -= n8;
@@ -303,8 +299,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
                       const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj) {
   extern __shared__ uint4 gemv_ring[];
   constexpr int S = kGemvStages;
-  pdl_wait();  // the activations come from the previous launch
-  pdl_trigger();
   // blocks of the first grid row take the shared expert (when there is one):
   // they start first, and their weight stream runs beside the routed blocks'
   int e = blockIdx.y;
@@ -394,7 +388,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
 cudaError_t launch_prep(const void* act, int rows, int K, const int32_t* gsrc, int gk, void* act16,
                         cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  return launch_after_previous(w4a16_prep_kernel, dim3(rows), dim3(128), 0, stream,
+  return launch_kernel(w4a16_prep_kernel, dim3(rows), dim3(128), 0, stream,
                                static_cast<const __nv_bfloat16*>(act), K / 8, gsrc, gk, static_cast<uint4*>(act16));
 }
 
@@ -405,7 +399,7 @@ cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, 
   const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
   const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
   if (grid.y == 0) return cudaSuccess;  // no routed expert and no shared expert in this call
-  return launch_after_previous(w4a16_gemv_kernel<F32OUT>, grid, dim3(kGemvWarps * 32), kGemvSmem, stream,
+  return launch_kernel(w4a16_gemv_kernel<F32OUT>, grid, dim3(kGemvWarps * 32), kGemvSmem, stream,
                                static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
                                static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
 }
@@ -435,7 +429,7 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
   const long long n8 = static_cast<long long>(rows) * (I / 8);
   const long long n8s = gu_shared != nullptr ? static_cast<long long>(T) * (Is / 8) : 0;
   if (n8 + n8s > 0) {
-    cudaError_t e = launch_after_previous(w4a16_prep_swiglu_kernel, dim3(static_cast<unsigned>((n8 + n8s + 255) / 256)),
+    cudaError_t e = launch_kernel(w4a16_prep_swiglu_kernel, dim3(static_cast<unsigned>((n8 + n8s + 255) / 256)),
                                           dim3(256), 0, stream, gu, I, n8, cfg.swiglu_limit,
                                           static_cast<uint4*>(act16), gu_shared, Is, n8s,
                                           static_cast<__nv_bfloat16*>(h_shared));
