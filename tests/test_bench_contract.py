@@ -6,9 +6,11 @@ listed by the committed ncu launch lists), the bytes a W4A16 expert holds
 weights), and the rule that a DRAM traffic figure is reported only while the
 profiled kernel source is unchanged."""
 
+import datetime
 import hashlib
 import json
 import os
+import sys
 
 import pytest
 
@@ -78,3 +80,28 @@ def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch)
     assert bench.traffic_from_profile("grouped_ffn_y") is None
     src.write_bytes(b"// kernel v2\n")  # the kernel changed after the capture
     assert bench.traffic_from_profile("grouped_ffn_x") is None
+
+
+def test_clock_sampler_drains_a_pipe_larger_than_its_buffer():
+    """The sampler reads its nvidia-smi child's output as it comes: a run
+    longer than a pipe buffer's worth of samples neither stalls the child
+    nor loses the later samples, and finish() returns promptly."""
+    import subprocess
+    import threading
+    import time
+
+    line = "2026/12/03 10:00:00.000, 1965, 1965, Not Active, Not Active, Not Active, Active"
+    n = 20000  # about 1.7 MB: far more than a 64 KB pipe buffer
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.lines, c.windows = [], []
+    c.proc = subprocess.Popen([sys.executable, "-c", f"import sys\nfor _ in range({n}): print({line!r})"],
+                              stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    c.reader = threading.Thread(target=c._drain, daemon=True)
+    c.reader.start()
+    assert c.proc.wait(timeout=60) == 0  # the child never blocks on a full pipe
+    ts = datetime.datetime.strptime(line.split(",")[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+    c.mark(ts - 1, ts + 1)
+    t0 = time.time()
+    res = c.finish()
+    assert time.time() - t0 < 15
+    assert res["samples"] == n and res["sm_mhz"] == 1965.0 and res["reasons"] == ["sw_power_cap"]
