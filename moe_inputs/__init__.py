@@ -11,13 +11,19 @@ and shared weights ~N(0, 1/fan_in) in bf16 (fan_in = hidden for gate/up and
 the router, intermediate for down), fp32 router weights ~N(0, 1/hidden),
 correction bias ~U(-b, b), and for the W4A16 layer uint4 codes ~U{0..15}
 packed two per byte (low nibble = even k) with bf16 per-group scales
-~U(0.005, 0.02), group 128 along K.
+~U(0.005, 0.02), group 128 along K.  NVFP4 layers (not one of the five):
+e2m1 codes ~U{0..15} packed the same way, one FP8 E4M3 scale byte per 16
+along K drawn uniformly from 0x30..0x3F (the E4M3 values 0.5 .. 1.875), and
+one fp32 scale per expert and projection ~U(0.25, 0.35) / sqrt(fan_in) --
+the bytes are drawn, never decoded, here.
 
 Draw order (one ``torch.Generator`` per device):
   CPU generator, seed s:    x, router weight, correction bias
   weight-device generator,  seed s + 1:
                             routed gate/up, routed down, shared gate/up,
-                            shared down  (W4A16: codes and scales per tensor)
+                            shared down  (W4A16: codes and scales per tensor;
+                            NVFP4: codes, scale bytes and fp32 scales per
+                            tensor)
 
 The routed/shared weights come from a generator on ``weight_device`` so the
 multi-GB layers can be drawn on the GPU in well under a second; their values
@@ -48,10 +54,12 @@ class LayerInputs:
     correction_bias: torch.Tensor   # [E] fp32
     w_gate_up: torch.Tensor         # bf16 [E, 2I, H]  | uint8 [E, 2I, H/2]
     w_down: torch.Tensor            # bf16 [E, H, I]   | uint8 [E, H, I/2]
-    s_gate_up: Optional[torch.Tensor]  # bf16 [E, 2I, H/128] (W4A16 only)
-    s_down: Optional[torch.Tensor]     # bf16 [E, H, I/128]  (W4A16 only)
+    s_gate_up: Optional[torch.Tensor]  # bf16 [E, 2I, H/128] (W4A16) | uint8 [E, 2I, H/16] (NVFP4)
+    s_down: Optional[torch.Tensor]     # bf16 [E, H, I/128]  (W4A16) | uint8 [E, H, I/16]  (NVFP4)
     shared_w_gate_up: Optional[torch.Tensor]  # bf16 [2I_s, H]
     shared_w_down: Optional[torch.Tensor]     # bf16 [H, I_s]
+    g_gate_up: Optional[torch.Tensor] = None  # fp32 [E] (NVFP4 only)
+    g_down: Optional[torch.Tensor] = None     # fp32 [E] (NVFP4 only)
 
     def to(self, device) -> "LayerInputs":
         def mv(t):
@@ -62,7 +70,8 @@ class LayerInputs:
             w_gate_up=mv(self.w_gate_up), w_down=mv(self.w_down),
             s_gate_up=mv(self.s_gate_up), s_down=mv(self.s_down),
             shared_w_gate_up=mv(self.shared_w_gate_up),
-            shared_w_down=mv(self.shared_w_down))
+            shared_w_down=mv(self.shared_w_down),
+            g_gate_up=mv(self.g_gate_up), g_down=mv(self.g_down))
 
 
 def _normal(shape, std, gen, device, dtype=torch.bfloat16):
@@ -115,11 +124,26 @@ def make_layer(cfg: LayerConfig, seed: int = 0, weight_device="cpu",
     dev = torch.device(weight_device)
     g = torch.Generator(device=dev).manual_seed(seed + 1)
     E, H, I, Is = cfg.E, cfg.H, cfg.I, cfg.I_s
-    if cfg.w4a16:
-        def codes(shape):
-            # two independent U{0..15} nibbles == one uniform byte
-            t = torch.empty(shape, dtype=torch.uint8, device=dev)
-            return t.random_(0, 256, generator=g)
+    g_gu = g_d = None
+
+    def codes(shape):
+        # two independent U{0..15} nibbles == one uniform byte
+        t = torch.empty(shape, dtype=torch.uint8, device=dev)
+        return t.random_(0, 256, generator=g)
+
+    def scale_bytes(shape):
+        t = torch.empty(shape, dtype=torch.uint8, device=dev)
+        return t.random_(0x30, 0x40, generator=g)
+
+    if cfg.nvfp4:
+        q_gu = codes((E, 2 * I, H // 2))
+        s_gu = scale_bytes((E, 2 * I, H // 16))
+        g_gu = _uniform((E,), 0.25 / math.sqrt(H), 0.35 / math.sqrt(H), g, dev)
+        q_d = codes((E, H, I // 2))
+        s_d = scale_bytes((E, H, I // 16))
+        g_d = _uniform((E,), 0.25 / math.sqrt(I), 0.35 / math.sqrt(I), g, dev)
+        w_gu, w_d = q_gu, q_d
+    elif cfg.w4a16:
         q_gu = codes((E, 2 * I, H // 2))
         s_gu = _uniform((E, 2 * I, H // 128), 0.005, 0.02, g, dev, torch.bfloat16)
         q_d = codes((E, H, I // 2))
@@ -134,4 +158,4 @@ def make_layer(cfg: LayerConfig, seed: int = 0, weight_device="cpu",
         sd = _normal((H, Is), 1.0 / math.sqrt(Is), g, dev)
     else:
         sgu = sd = None
-    return LayerInputs(cfg, x, router_w, bias, w_gu, w_d, s_gu, s_d, sgu, sd)
+    return LayerInputs(cfg, x, router_w, bias, w_gu, w_d, s_gu, s_d, sgu, sd, g_gu, g_d)

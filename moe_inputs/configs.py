@@ -35,6 +35,7 @@ class LayerConfig:
     zipf_s: float = 1.2
     bias_scale: float = 0.0
     w4a16: bool = False
+    nvfp4: bool = False         # NVFP4 routed experts (e2m1 codes, e4m3 scale per 16, fp32 per expert)
     x_scale: float = 1.0        # x ~ N(0, x_scale^2) (1 in every benchmark layer)
 
     @property
@@ -64,4 +65,10 @@ PREFILL_W4A16 = LayerConfig("prefill_w4a16", T=16384, H=6144, E=256, k=8, I=2048
                             I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
                             w4a16=True)
 
-CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16, PREFILL_W4A16)}
+# Not one of the five benchmark layers either: the same shape with NVFP4
+# expert weights (the routed NVFP4 MoE the module summary names).
+PREFILL_NVFP4 = LayerConfig("prefill_nvfp4", T=16384, H=6144, E=256, k=8, I=2048,
+                            I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
+                            nvfp4=True)
+
+CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16, PREFILL_W4A16, PREFILL_NVFP4)}

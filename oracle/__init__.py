@@ -6,7 +6,7 @@ and the passages each one follows.
 """
 
 from .moe_oracle import (  # noqa: F401
-    LayerResult, Permutation, Selection, dequant_int4_g128, expert_ffn,
+    LayerResult, Permutation, Selection, dequant_int4_g128, dequant_nvfp4, e2m1_value, e4m3_value, expert_ffn,
     expert_hidden, expert_weights64, moe_forward, moe_partial, override_selection, permute, router_logits,
     select_topk, sigmoid, swiglu_clamped,
 )

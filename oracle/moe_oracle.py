@@ -33,6 +33,13 @@ Readings where the pages are silent (each also listed in the design notes):
   * gate rows come first in the fused gate/up weight ([0, I) gate, [I, 2I) up);
   * W4A16: two uint4 codes per byte along K, low nibble = even k, zero point
     8, one bf16 scale per (output row, 128-wide K group): w = (q - 8) * scale.
+  * NVFP4 (the module summary's "routed NVFP4 MoE"; the pages give no
+    layout): FP4 E2M1 codes packed as for W4A16, one FP8 E4M3 scale per
+    (output row, 16-wide K block), and one fp32 scale per expert and weight
+    tensor (the fused gate/up is one tensor):
+    w = e2m1(code) * e4m3(block scale) * tensor scale.  The element formats
+    are the OCP ones: E2M1 of the Microscaling Formats (MX) v1.0
+    specification, E4M3 of the OCP 8-bit Floating Point specification.
 
 Pins: tests/test_oracle.py checks every function here against hand-worked
 closed forms (tests/golden/), brute-force enumeration, invariants and
@@ -176,6 +183,50 @@ def dequant_int4_g128(q: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
     return (codes - 8.0) * sc
 
 
+def e2m1_value(code: torch.Tensor) -> torch.Tensor:
+    """FP4 E2M1 (OCP Microscaling Formats v1.0): bit 3 sign, bits 2..1
+    exponent with bias 1, bit 0 mantissa.  Exponent field 0 is subnormal,
+    m * 2^-1 (0 or 0.5); otherwise (1 + m / 2) * 2^(e - 1).  The format has
+    no infinity and no NaN.  code: integer tensor of 4-bit values -> fp64."""
+    c = code.to(torch.int64)
+    sign = (c >> 3) & 1
+    e = ((c >> 1) & 3).to(f64)
+    m = (c & 1).to(f64)
+    mag = torch.where(e == 0, m * 0.5, (1.0 + m / 2.0) * torch.pow(2.0, e - 1.0))
+    return torch.where(sign == 1, -mag, mag)
+
+
+def e4m3_value(b: torch.Tensor) -> torch.Tensor:
+    """FP8 E4M3 (OCP 8-bit Floating Point): bit 7 sign, bits 6..3 exponent
+    with bias 7, bits 2..0 mantissa.  Exponent field 0 is subnormal,
+    (m / 8) * 2^-6; otherwise (1 + m / 8) * 2^(e - 7).  No infinity; the two
+    patterns S.1111.111 are NaN.  b: uint8 tensor -> fp64."""
+    c = b.to(torch.int64)
+    sign = (c >> 7) & 1
+    e = ((c >> 3) & 15).to(f64)
+    m = (c & 7).to(f64)
+    mag = torch.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * torch.pow(2.0, e - 7.0))
+    mag = torch.where((e == 15) & (m == 7), torch.full_like(mag, float("nan")), mag)
+    return torch.where(sign == 1, -mag, mag)
+
+
+def dequant_nvfp4(q: torch.Tensor, block_scale: torch.Tensor, tensor_scale) -> torch.Tensor:
+    """NVFP4 weight: w[n, k] = e2m1(code[n, k]) * e4m3(block_scale[n, k // 16])
+    * tensor_scale, with the codes of byte q[n, c] at k = 2c (low nibble) and
+    k = 2c + 1 (high nibble).  q: uint8 [N, K/2], block_scale: uint8
+    [N, K/16] (E4M3 bit patterns), tensor_scale: fp32 scalar -> fp64 [N, K]."""
+    q = q.detach().cpu()
+    N, half = q.shape
+    K = 2 * half
+    lo = e2m1_value(q & 0xF)
+    hi = e2m1_value(q >> 4)
+    vals = torch.stack([lo, hi], dim=-1).reshape(N, K)
+    sc = e4m3_value(block_scale.detach().cpu()).repeat_interleave(16, dim=1)
+    assert sc.shape == (N, K)
+    g = float(torch.as_tensor(tensor_scale, dtype=torch.float32))
+    return vals * sc * g
+
+
 def expert_ffn(v: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
                limit: float) -> torch.Tensor:
     """FFN(v) = W_down (silu(min(W_gate v, L)) * clamp(W_up v, -L, L)).
@@ -198,6 +249,9 @@ def expert_hidden(v, w_gate_up, limit):
 
 def expert_weights64(layer, e: int):
     """Routed expert e's (w_gate_up [2I, H], w_down [H, I]) in fp64."""
+    if getattr(layer.cfg, "nvfp4", False):
+        return (dequant_nvfp4(layer.w_gate_up[e], layer.s_gate_up[e], layer.g_gate_up[e].cpu()),
+                dequant_nvfp4(layer.w_down[e], layer.s_down[e], layer.g_down[e].cpu()))
     if layer.cfg.w4a16:
         return (dequant_int4_g128(layer.w_gate_up[e], layer.s_gate_up[e]),
                 dequant_int4_g128(layer.w_down[e], layer.s_down[e]))

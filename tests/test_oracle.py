@@ -30,6 +30,12 @@ def hand(golden_dir):
         return json.load(f)
 
 
+@pytest.fixture(scope="module")
+def hand_nvfp4(golden_dir):
+    with open(os.path.join(golden_dir, "nvfp4_hand.json")) as f:
+        return json.load(f)
+
+
 def _s(z):
     return 1.0 / (1.0 + math.exp(-z))
 
@@ -132,6 +138,90 @@ def test_dequant_group_index():
     W = oracle.dequant_int4_g128(q, s)
     assert (W[0, :128] == 1).all() and (W[0, 128:] == 2).all()
     assert (W[1, :128] == 4).all() and (W[1, 128:] == 8).all()
+
+
+# ------------------------------------------------------------------- NVFP4 --
+
+def test_e2m1_table(hand_nvfp4):
+    """Every FP4 E2M1 code against the format's value set (and its sign bit)."""
+    got = oracle.e2m1_value(torch.arange(16))
+    assert got.tolist() == hand_nvfp4["e2m1_by_code"]
+    assert (torch.signbit(got[8:])).all() and not torch.signbit(got[:8]).any()
+
+
+def test_e4m3_matches_torch_float8():
+    """All 256 E4M3 bit patterns against torch's float8_e4m3fn conversion
+    (a library routine), NaN exactly at S.1111.111."""
+    b = torch.arange(256, dtype=torch.int64).to(torch.uint8)
+    got = oracle.e4m3_value(b)
+    lib = b.view(torch.float8_e4m3fn).to(f64)
+    assert torch.equal(torch.isnan(got), torch.isnan(lib))
+    assert torch.isnan(got).nonzero().flatten().tolist() == [0x7F, 0xFF]
+    ok = ~torch.isnan(lib)
+    assert torch.equal(got[ok], lib[ok])
+
+
+def test_e4m3_hand_values(hand_nvfp4):
+    sp = hand_nvfp4["e4m3_spot"]
+    got = oracle.e4m3_value(torch.tensor(sp["bytes"], dtype=torch.int64).to(torch.uint8))
+    assert got.tolist() == sp["values"]
+    assert torch.isnan(oracle.e4m3_value(torch.tensor(sp["nan_bytes"], dtype=torch.int64).to(torch.uint8))).all()
+
+
+def test_hand_nvfp4_dequant(hand_nvfp4):
+    d = hand_nvfp4["dequant"]
+    q = torch.zeros(1, 16, dtype=torch.uint8)
+    for c, v in d["q_bytes"].items():
+        q[0, int(c)] = v
+    bs = torch.tensor([d["block_scale_bytes"]], dtype=torch.uint8)
+    W = oracle.dequant_nvfp4(q, bs, torch.tensor(d["tensor_scale"], dtype=torch.float32))
+    want = torch.zeros(1, 32, dtype=f64)
+    for k, v in d["w_nonzero"].items():
+        want[0, int(k)] = v
+    assert W.shape == (1, 32)
+    assert torch.equal(W, want)
+
+
+def test_nvfp4_block_index():
+    """Block scale b covers k in [16b, 16b + 16) of its own row only."""
+    q = torch.full((2, 32), 0x22, dtype=torch.uint8)          # code 2 (= 1.0) everywhere
+    bs = torch.tensor([[0x38, 0x40, 0x48, 0x50], [0x30, 0x28, 0x20, 0x18]], dtype=torch.uint8)
+    W = oracle.dequant_nvfp4(q, bs, 1.0)
+    want_row = [[1.0, 2.0, 4.0, 8.0], [0.5, 0.25, 0.125, 0.0625]]
+    for n in range(2):
+        for b in range(4):
+            assert (W[n, 16 * b:16 * b + 16] == want_row[n][b]).all()
+
+
+def test_nvfp4_layer_reduces_to_bf16_layer(hand_nvfp4):
+    """An NVFP4 layer with power-of-two tensor scales gives the same output
+    as the bf16 layer holding its weights, formed here from the E2M1 value
+    table and torch's float8_e4m3fn (e2m1 x e4m3 has at most 6 significant
+    bits, exact in bf16)."""
+    cfg = LayerConfig("fp4", T=6, H=256, E=3, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
+                      nvfp4=True)
+    g = torch.Generator().manual_seed(4)
+    base = moe_inputs.make_layer(cfg.with_(nvfp4=False), seed=9)
+    table = torch.tensor(hand_nvfp4["e2m1_by_code"], dtype=f64)
+
+    def pack(E, N, K):
+        codes = torch.randint(0, 16, (E, N, K), generator=g, dtype=torch.int64)
+        sb = torch.randint(0x20, 0x48, (E, N, K // 16), generator=g, dtype=torch.int64).to(torch.uint8)
+        ts = 2.0 ** (-torch.randint(3, 7, (E,), generator=g)).to(torch.float32)
+        w = (table[codes] * sb.view(torch.float8_e4m3fn).to(f64).repeat_interleave(16, dim=2)
+             * ts.to(f64)[:, None, None])
+        q = (codes[..., 0::2] | (codes[..., 1::2] << 4)).to(torch.uint8)
+        return q, sb, ts, w.to(torch.bfloat16)
+
+    qgu, sgu, tgu, wgu = pack(cfg.E, 2 * cfg.I, cfg.H)
+    qd, sd, td, wd = pack(cfg.E, cfg.H, cfg.I)
+    lay4 = LayerInputs(cfg, base.x, base.router_w, base.correction_bias, qgu, qd, sgu, sd,
+                       base.shared_w_gate_up, base.shared_w_down, tgu, td)
+    lay16 = LayerInputs(cfg.with_(nvfp4=False), base.x, base.router_w, base.correction_bias,
+                        wgu, wd, None, None, base.shared_w_gate_up, base.shared_w_down)
+    a, b = oracle.moe_forward(lay4), oracle.moe_forward(lay16)
+    assert (a.selection.ids == b.selection.ids).all()
+    assert torch.allclose(a.out, b.out, rtol=1e-12, atol=1e-12)
 
 
 # ------------------------------------------------------------- brute force --

@@ -72,6 +72,43 @@ def _dequant_hi_first(q, scale):
     return (codes - 8.0) * om._cpu64(scale).repeat_interleave(128, dim=1)
 
 
+def _nvfp4_hi_first(q, block_scale, tensor_scale):      # high nibble taken as the even k
+    q = q.detach().cpu()
+    N, half = q.shape
+    vals = torch.stack([om.e2m1_value(q >> 4), om.e2m1_value(q & 0xF)], -1).reshape(N, 2 * half)
+    sc = om.e4m3_value(block_scale.detach().cpu()).repeat_interleave(16, dim=1)
+    return vals * sc * float(tensor_scale)
+
+
+def _nvfp4_block32(q, block_scale, tensor_scale):       # one scale per 32 instead of 16
+    q = q.detach().cpu()
+    N, half = q.shape
+    vals = torch.stack([om.e2m1_value(q & 0xF), om.e2m1_value(q >> 4)], -1).reshape(N, 2 * half)
+    sc = om.e4m3_value(block_scale.detach().cpu()).repeat_interleave(32, dim=1)[:, :2 * half]
+    return vals * sc * float(tensor_scale)
+
+
+def _nvfp4_no_tensor_scale(q, block_scale, tensor_scale):
+    return _orig_nvfp4(q, block_scale, 1.0)
+
+
+def _e2m1_bias0(code):                                   # exponent bias 0 instead of 1
+    return 2.0 * _orig_e2m1(code)
+
+
+def _e2m1_no_subnormal(code):                            # exponent field 0 read as normal
+    c = code.to(torch.int64)
+    v = _orig_e2m1(code)
+    sub = ((c >> 1) & 3) == 0
+    fixed = torch.where((c & 1) == 1, torch.full_like(v, 0.75), torch.full_like(v, 0.5))
+    fixed = torch.where(((c >> 3) & 1) == 1, -fixed, fixed)
+    return torch.where(sub, fixed, v)
+
+
+def _e4m3_bias8(b):                                      # exponent bias 8 instead of 7
+    return 0.5 * _orig_e4m3(b)
+
+
 def _ffn_down_transposed(v, w_gate_up, w_down, limit):
     I = w_down.shape[1]
     gu = v @ w_gate_up.T
@@ -80,6 +117,9 @@ def _ffn_down_transposed(v, w_gate_up, w_down, limit):
 
 
 _orig_select = om.select_topk
+_orig_nvfp4 = om.dequant_nvfp4
+_orig_e2m1 = om.e2m1_value
+_orig_e4m3 = om.e4m3_value
 
 
 def _expect_fail(fn, *args):
@@ -120,6 +160,44 @@ def test_renorm_after_alpha_is_caught(monkeypatch, hand):
 def test_nibble_order_is_caught(monkeypatch, hand):
     _patch(monkeypatch, "dequant_int4_g128", _dequant_hi_first)
     _expect_fail(pins.test_hand_w4a16_dequant, hand)
+
+
+def test_nvfp4_nibble_order_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "dequant_nvfp4", _nvfp4_hi_first)
+    _expect_fail(pins.test_hand_nvfp4_dequant, hand_nvfp4)
+
+
+def test_nvfp4_block_of_32_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "dequant_nvfp4", _nvfp4_block32)
+    _expect_fail(pins.test_nvfp4_block_index)
+
+
+def test_nvfp4_dropped_tensor_scale_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "dequant_nvfp4", _nvfp4_no_tensor_scale)
+    _expect_fail(pins.test_hand_nvfp4_dequant, hand_nvfp4)
+
+
+def test_nvfp4_layer_dispatch_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "dequant_nvfp4", _nvfp4_no_tensor_scale)
+    _expect_fail(pins.test_nvfp4_layer_reduces_to_bf16_layer, hand_nvfp4)
+
+
+def test_e2m1_wrong_bias_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "e2m1_value", _e2m1_bias0)
+    _expect_fail(pins.test_e2m1_table, hand_nvfp4)
+    _expect_fail(pins.test_hand_nvfp4_dequant, hand_nvfp4)
+
+
+def test_e2m1_missing_subnormal_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "e2m1_value", _e2m1_no_subnormal)
+    _expect_fail(pins.test_e2m1_table, hand_nvfp4)
+
+
+def test_e4m3_wrong_bias_is_caught(monkeypatch, hand_nvfp4):
+    _patch(monkeypatch, "e4m3_value", _e4m3_bias8)
+    _expect_fail(pins.test_e4m3_matches_torch_float8)
+    _expect_fail(pins.test_e4m3_hand_values, hand_nvfp4)
+    _expect_fail(pins.test_hand_nvfp4_dequant, hand_nvfp4)
 
 
 def test_transposed_down_is_caught(monkeypatch):
@@ -173,6 +251,7 @@ def test_override_without_renorm_is_caught(monkeypatch, hand):
 
 
 hand = pins.hand
+hand_nvfp4 = pins.hand_nvfp4
 
 
 def test_partial_with_inclusive_range_is_caught(monkeypatch, tiny_layer, tiny_result):
