@@ -238,12 +238,13 @@ def w4a16_bytes(cfg, ids):
 def launches_per_step(cfg):
     """Kernels one forward launches: router 3 (weight split, tensor-core
     logits, top-k), permute 2 (count/rank with the scan in its last block,
-    then the scatter into x_perm, or for int4 experts the maps alone, their
+    then the scatter into x_perm, or for 4-bit experts the maps alone, their
     activation conversion gathering the rows), combine 1, plus the expert
     FFN path and the shared expert's launches when it does not ride in the
     routed ones."""
     n = 6
-    prefill = cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E   # int4 dequantised in shared memory, tensor cores
+    # 4-bit codes dequantised in shared memory, tensor cores (NVFP4 always)
+    prefill = cfg.nvfp4 or (cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E)
     gemv = cfg.w4a16 and not prefill                      # int4 dequantised in registers
     shared = 0
     if cfg.I_s > 0:
@@ -251,7 +252,7 @@ def launches_per_step(cfg):
             shared = 0      # in the two GEMV launches
         elif cfg.T <= 32:
             shared = 4      # split-K GEMMs + ordered slice sums
-        elif cfg.w4a16:
+        elif cfg.w4a16 or cfg.nvfp4:
             shared = 2      # its own tcgen05 gate/up and down launches
         else:
             shared = 0      # one more problem of the routed tcgen05 launches
@@ -263,8 +264,9 @@ def launches_per_step(cfg):
 
 
 def base_line(args, n_gpus, cfg):
+    bytes_per_weight = 0.5 + 1 / 16 if cfg.nvfp4 else 0.5 + 2 / 128 if cfg.w4a16 else 2
     l2 = ("inputs larger than L2 (expert weights streamed per step: %.2f GB)"
-          % ((cfg.E * 3 * cfg.H * cfg.I * (0.5 if cfg.w4a16 else 2) + 6 * cfg.H * cfg.I_s) / 1e9))
+          % ((cfg.E * 3 * cfg.H * cfg.I * bytes_per_weight + 6 * cfg.H * cfg.I_s) / 1e9))
     return {
         "metric": METRIC, "unit": "tokens/s", "n_gpus": n_gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
@@ -331,7 +333,8 @@ def measure_decode(dev, iters, clocks, max_over_ranks):
                          router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias),
                          w_gate_up=mv(inp.w_gate_up), w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up),
                          s_down=mv(inp.s_down), shared_w_gate_up=mv(inp.shared_w_gate_up),
-                         shared_w_down=mv(inp.shared_w_down), max_tokens=c.T)
+                         shared_w_down=mv(inp.shared_w_down), g_gate_up=mv(inp.g_gate_up),
+                         g_down=mv(inp.g_down), max_tokens=c.T)
     x = inp.x.to(dev)
     T, k, E, H = c.T, c.k, c.E, c.H
     R = T * k
@@ -404,7 +407,8 @@ def bench_ours(args, rank, world, local_rank):
                          router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias),
                          w_gate_up=mv(inp.w_gate_up), w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up),
                          s_down=mv(inp.s_down), shared_w_gate_up=mv(inp.shared_w_gate_up),
-                         shared_w_down=mv(inp.shared_w_down), max_tokens=c.T)
+                         shared_w_down=mv(inp.shared_w_down), g_gate_up=mv(inp.g_gate_up),
+                         g_down=mv(inp.g_down), max_tokens=c.T)
     x = inp.x.to(dev)
     out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -447,7 +451,7 @@ def bench_ours(args, rank, world, local_rank):
 
     # --- per-stage durations (the kernels the forward launches, one C-ABI call
     # per stage, events between).  As in moe_forward: bf16 experts permute
-    # into x_perm; int4 experts write the maps only and gather in the FFN.
+    # into x_perm; 4-bit experts write the maps only and gather in the FFN.
     T, k, E, H = c.T, c.k, c.E, c.H
     R = T * k
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
@@ -456,7 +460,7 @@ def bench_ours(args, rank, world, local_rank):
     row_of = torch.empty(R, dtype=torch.int32, device=dev)
     src = torch.empty(R, dtype=torch.int32, device=dev)
     w_perm = torch.empty(R, dtype=torch.float32, device=dev)
-    x_perm = None if c.w4a16 else torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    x_perm = None if (c.w4a16 or c.nvfp4) else torch.empty(R, H, dtype=torch.bfloat16, device=dev)
 
     def permute():
         rse.moe_permute(layer.cfg, ids, tw, x, T, offs, row_of, src, w_perm, x_perm, layer.ws)
@@ -568,6 +572,9 @@ def bench_ours(args, rank, world, local_rank):
         achieved = (routed_f + shared_f) / ffn_s / 1e12
         roof = {"kernel": ("grouped W4A16 FFN (int4 dequantised to fp16 in shared memory, tcgen05 gate/up+SwiGLU "
                            "and down+weight launches) + bf16 shared expert") if c.w4a16 else
+                          ("grouped NVFP4 FFN (E2M1 x E4M3 dequantised to fp16 in shared memory, tcgen05 "
+                           "gate/up+SwiGLU and down+weight launches, fp32 tensor scales in the epilogues) + bf16 "
+                           "shared expert") if c.nvfp4 else
                           "grouped SwiGLU FFN (tcgen05 gate/up+SwiGLU and down+weight launches, "
                           "routed + shared expert)",
                 "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -631,6 +638,7 @@ def bench_ep(args, rank, world, local_rank):
         router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias), w_gate_up=mv(inp.w_gate_up),
         w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up), s_down=mv(inp.s_down),
         shared_w_gate_up=mv(inp.shared_w_gate_up), shared_w_down=mv(inp.shared_w_down),
+        g_gate_up=mv(inp.g_gate_up), g_down=mv(inp.g_down),
         rank=rank, world=world, max_tokens=c.T, group=group)
     x = inp.x.to(dev)
     out = torch.empty(c.T, c.H, dtype=torch.bfloat16, device=dev)

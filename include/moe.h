@@ -31,8 +31,9 @@
  *   - Arguments are validated on the host before anything is launched; a
  *     non-OK status means nothing was enqueued.
  *   - Row-major layouts; bf16 is IEEE bfloat16 stored as uint16.
- *   - Data pointers must be 16-byte aligned; H, I and I_s multiples of 8
- *     (16-byte rows); the W4A16 format needs H and I multiples of 128.
+ *   - Data pointers must be 16-byte aligned (the NVFP4 tensor scales: 4
+ *     bytes); H, I and I_s multiples of 8 (16-byte rows); the W4A16 and
+ *     NVFP4 formats need H and I multiples of 128.
  *   - T == 0 returns MOE_OK and launches nothing.
  *   - `ws` is a caller-owned device workspace of at least
  *     moe_workspace_size(cfg, T) bytes, 256-byte aligned, whose first 256
@@ -69,7 +70,9 @@ typedef enum moe_status {
 
 typedef enum moe_weight_format {
   MOE_W_BF16 = 0,        /* routed expert weights in bf16 */
-  MOE_W_INT4_G128 = 1    /* W4A16: uint4 codes, bf16 scale per 128 along K */
+  MOE_W_INT4_G128 = 1,   /* W4A16: uint4 codes, bf16 scale per 128 along K */
+  MOE_W_NVFP4 = 2        /* NVFP4: E2M1 codes, E4M3 scale per 16 along K,
+                            fp32 scale per expert weight tensor */
 } moe_weight_format;
 
 /* Largest k the router kernel selects per token ([glm5next] constant
@@ -88,8 +91,8 @@ typedef struct moe_config {
   int32_t shared_inter;          /* I_s (multiple of 8; 0 = no shared expert) */
   float swiglu_limit;            /* L > 0, required (no default); +inf = no
                                     clamp.  gate <- min(gate, L),
-                                    up <- clamp(up, -L, L).  W4A16 experts:
-                                    L <= MOE_INT4_MAX_SWIGLU_LIMIT */
+                                    up <- clamp(up, -L, L).  W4A16 and NVFP4
+                                    experts: L <= MOE_INT4_MAX_SWIGLU_LIMIT */
   float routed_scaling_factor;   /* alpha: multiplies the routed weights; the
                                     shared expert is added unscaled */
   int32_t renormalize;           /* 1: divide the k unbiased scores by their
@@ -102,12 +105,15 @@ typedef struct moe_config {
 typedef struct moe_weights {
   const float* router_w;         /* fp32 [E, H] */
   const float* correction_bias;  /* fp32 [E], or NULL for zero bias */
-  const void* w_gate_up;         /* bf16 [E, 2I, H]  | uint8 [E, 2I, H/2] */
-  const void* s_gate_up;         /* NULL             | bf16  [E, 2I, H/128] */
-  const void* w_down;            /* bf16 [E, H, I]   | uint8 [E, H, I/2] */
-  const void* s_down;            /* NULL             | bf16  [E, H, I/128] */
-  const void* shared_w_gate_up;  /* bf16 [2I_s, H] (NULL iff I_s == 0) */
-  const void* shared_w_down;     /* bf16 [H, I_s]  (NULL iff I_s == 0) */
+  /*                                bf16            | W4A16                  | NVFP4 */
+  const void* w_gate_up;         /* bf16 [E, 2I, H] | uint8 [E, 2I, H/2]     | uint8 [E, 2I, H/2] */
+  const void* s_gate_up;         /* NULL            | bf16  [E, 2I, H/128]   | E4M3 uint8 [E, 2I, H/16] */
+  const void* w_down;            /* bf16 [E, H, I]  | uint8 [E, H, I/2]      | uint8 [E, H, I/2] */
+  const void* s_down;            /* NULL            | bf16  [E, H, I/128]    | E4M3 uint8 [E, H, I/16] */
+  const void* shared_w_gate_up;  /* bf16 [2I_s, H] (NULL iff I_s == 0), every format */
+  const void* shared_w_down;     /* bf16 [H, I_s]  (NULL iff I_s == 0), every format */
+  const float* g_gate_up;        /* NVFP4: fp32 [E] tensor scale of each gate/up weight; else ignored */
+  const float* g_down;           /* NVFP4: fp32 [E] tensor scale of each down weight; else ignored */
 } moe_weights;
 /* W4A16 (int4) packing: byte q[n, c] holds the codes of k = 2c (low nibble)
  * and k = 2c + 1 (high nibble); w[n, k] = (code - 8) * scale[n, k / 128].
@@ -128,6 +134,16 @@ typedef struct moe_weights {
  * The benchmark layers (x ~ N(0, 1), scales in [0.005, 0.02], L = 7) sit far
  * inside these bounds. */
 #define MOE_INT4_MAX_SWIGLU_LIMIT 255.0f
+
+/* NVFP4 packing ([glm5next] module summary: routed NVFP4 MoE; element
+ * formats of the OCP specifications: FP4 E2M1 of Microscaling Formats v1.0,
+ * FP8 E4M3 of 8-bit Floating Point): byte q[n, c] holds the E2M1 codes of
+ * k = 2c (low nibble) and k = 2c + 1 (high nibble);
+ *   w[n, k] = e2m1(code) * e4m3(s[n, k / 16]) * g[e].
+ * The grouped tensor-core GEMM forms e2m1 * e4m3 in fp16, which is exact for
+ * every finite E4M3 scale (the E4M3 NaN patterns give NaN weights), and
+ * multiplies the fp32 accumulators by g[e]; the activation limits of the
+ * W4A16 range note above (fp16 x and h, swiglu_limit) hold as stated there. */
 
 /* Human-readable name of a status.  Never NULL. */
 MOE_API const char* moe_status_string(moe_status status);
@@ -192,8 +208,10 @@ MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids,
  * run the W4A16 GEMV kernels that dequantise in registers ([glm5next]
  * W4A16_GEMV_MODULE) when there are fewer than 32 routed rows per expert on
  * average, else a grouped tensor-core GEMM that dequantises the int4 codes
- * into fp16 tiles in shared memory ([glm5next] MOE_GROUPED_MODULE); both
- * round h to bf16 as the bf16 path does.
+ * into fp16 tiles in shared memory ([glm5next] MOE_GROUPED_MODULE).
+ * MOE_W_NVFP4 weights always run that grouped tensor-core GEMM, with E2M1
+ * codes and E4M3 block scales decoded into the fp16 tiles.  Every format
+ * rounds h to bf16 as the bf16 path does.
  * When x_shared != NULL the shared expert runs in the same launches:
  *   shared_out[t] = bf16( SwiGLU_clamped FFN_shared(x_shared[t]) ), unscaled.
  *   x_perm          bf16 [T*k, H]    expert_offsets int32 [E+1]
@@ -210,7 +228,7 @@ MOE_API moe_status moe_grouped_swiglu_ffn(const moe_config* cfg, const moe_weigh
  * loads ([glm5next] MOE_MODULE token permute and forward_prefill_gemm): the
  * same result as moe_grouped_swiglu_ffn on x_perm[r] = x[src[r] / k], but
  * routed row r is read straight from token src[r] / k of x, so x_perm is
- * never written.  The int4 kernels gather while converting the activations
+ * never written.  The 4-bit kernels gather while converting the activations
  * to fp16 (the conversion pass they run anyway).  The bf16 tensor-core
  * kernel copies four token rows per TMA gather: correct, but on a B200 its
  * gate/up launch takes about twice as long as with the contiguous token
@@ -244,8 +262,9 @@ MOE_API moe_status moe_combine(const moe_config* cfg, const void* y_perm,
 /* The whole layer in one call: router -> permute -> grouped FFN (routed +
  * shared) -> combine, enqueued on `stream` with no host synchronisation.
  * bf16 experts: the permute writes x_perm into the workspace and the FFN
- * loads contiguous token boxes.  int4 experts: the permute writes the maps
- * only and the FFN gathers the rows as moe_grouped_swiglu_ffn_gather does.
+ * loads contiguous token boxes.  int4 and NVFP4 experts: the permute writes
+ * the maps only and the FFN gathers the rows as moe_grouped_swiglu_ffn_gather
+ * does.
  *   x    bf16 [T, H];  out bf16 [T, H]
  *   topk_ids_opt int32 [T, k] / topk_w_opt fp32 [T, k]: if non-NULL, the
  *   router's selection is also written there. */
@@ -272,7 +291,8 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const moe_weights* w,
  *         width of the shared intermediate (0: no shared work on this rank);
  *         cfg->num_experts is the full E (the router ranks every expert).
  *   w     router_w / correction_bias: the full [E, H] / [E];
- *         w_gate_up, w_down (and s_gate_up, s_down): the LOCAL experts only,
+ *         w_gate_up, w_down (and s_gate_up, s_down, g_gate_up, g_down):
+ *         the LOCAL experts only,
  *         [expert_end - expert_begin, ...], local expert 0 = global expert
  *         expert_begin (may be NULL when the range is empty);
  *         shared_w_gate_up [2 I_s_local, H] (the slice's gate rows, then its

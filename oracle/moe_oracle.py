@@ -218,10 +218,13 @@ def dequant_nvfp4(q: torch.Tensor, block_scale: torch.Tensor, tensor_scale) -> t
     q = q.detach().cpu()
     N, half = q.shape
     K = 2 * half
-    lo = e2m1_value(q & 0xF)
-    hi = e2m1_value(q >> 4)
+    # each format's values, evaluated once by the definitions above, then looked up
+    e2m1 = e2m1_value(torch.arange(16))
+    e4m3 = e4m3_value(torch.arange(256, dtype=torch.int64).to(torch.uint8))
+    lo = e2m1[(q & 0xF).long()]
+    hi = e2m1[(q >> 4).long()]
     vals = torch.stack([lo, hi], dim=-1).reshape(N, K)
-    sc = e4m3_value(block_scale.detach().cpu()).repeat_interleave(16, dim=1)
+    sc = e4m3[block_scale.detach().cpu().long()].repeat_interleave(16, dim=1)
     assert sc.shape == (N, K)
     g = float(torch.as_tensor(tensor_scale, dtype=torch.float32))
     return vals * sc * g

@@ -15,7 +15,7 @@ from typing import Optional
 from . import _abi
 from ._abi import (  # noqa: F401
     EXPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
-    MOE_ERR_WORKSPACE, MOE_MAX_EXPERTS, MOE_MAX_TOP_K, MOE_OK, MOE_W_BF16, MOE_W_INT4_G128, MoEError,
+    MOE_ERR_WORKSPACE, MOE_MAX_EXPERTS, MOE_MAX_TOP_K, MOE_OK, MOE_W_BF16, MOE_W_INT4_G128, MOE_W_NVFP4, MoEError,
     load_library, make_config, make_weights, moe_combine, moe_config, moe_config_validate, moe_forward,
     moe_grouped_swiglu_ffn, moe_grouped_swiglu_ffn_gather, moe_permute, moe_read_device_error, moe_router_topk,
     moe_weights,
@@ -33,14 +33,16 @@ class MoELayer:
     fp32 [E] or None; w_gate_up bf16 [E, 2I, H] (or uint8 [E, 2I, H/2] with
     s_gate_up bf16 [E, 2I, H/128]); w_down bf16 [E, H, I] (or uint8
     [E, H, I/2] with s_down bf16 [E, H, I/128]); shared_w_gate_up bf16
-    [2I_s, H] and shared_w_down bf16 [H, I_s] (None when I_s == 0)."""
+    [2I_s, H] and shared_w_down bf16 [H, I_s] (None when I_s == 0).
+    NVFP4 experts: uint8 E2M1 codes as above, s_gate_up / s_down uint8 E4M3
+    scales [E, 2I, H/16] / [E, H, I/16], and g_gate_up / g_down fp32 [E]
+    tensor scales (their presence selects the format)."""
 
     def __init__(self, *, hidden, num_experts, top_k, expert_inter, shared_inter, swiglu_limit,
                  routed_scaling_factor, renormalize, router_w, correction_bias, w_gate_up, w_down,
                  s_gate_up=None, s_down=None, shared_w_gate_up=None, shared_w_down=None,
-                 max_tokens: int = 0):
-        import torch
-        fmt = MOE_W_INT4_G128 if w_gate_up.dtype == torch.uint8 else MOE_W_BF16
+                 g_gate_up=None, g_down=None, max_tokens: int = 0):
+        fmt = _abi.weight_format(w_gate_up, g_gate_up)
         self.cfg = make_config(hidden, num_experts, top_k, expert_inter, shared_inter, swiglu_limit,
                                routed_scaling_factor, renormalize, fmt)
         st = moe_config_validate(self.cfg)
@@ -48,7 +50,8 @@ class MoELayer:
             raise MoEError(st, "moe_config_validate")
         self.tensors = dict(router_w=router_w, correction_bias=correction_bias, w_gate_up=w_gate_up,
                             s_gate_up=s_gate_up, w_down=w_down, s_down=s_down,
-                            shared_w_gate_up=shared_w_gate_up, shared_w_down=shared_w_down)
+                            shared_w_gate_up=shared_w_gate_up, shared_w_down=shared_w_down,
+                            g_gate_up=g_gate_up, g_down=g_down)
         self.w = make_weights(**self.tensors)
         self.device = router_w.device
         self.ws = None

@@ -25,6 +25,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 
 MOE_W_BF16 = 0
 MOE_W_INT4_G128 = 1
+MOE_W_NVFP4 = 2
 MOE_MAX_TOP_K = 16
 MOE_MAX_EXPERTS = 1024
 MOE_INT4_MAX_SWIGLU_LIMIT = 255.0
@@ -71,6 +72,8 @@ class moe_weights(ctypes.Structure):
         ("s_down", ctypes.c_void_p),
         ("shared_w_gate_up", ctypes.c_void_p),
         ("shared_w_down", ctypes.c_void_p),
+        ("g_gate_up", ctypes.c_void_p),
+        ("g_down", ctypes.c_void_p),
     ]
 
 
@@ -151,9 +154,20 @@ def make_config(hidden, num_experts, top_k, expert_inter, shared_inter, swiglu_l
 
 
 def make_weights(router_w=None, correction_bias=None, w_gate_up=None, s_gate_up=None, w_down=None,
-                 s_down=None, shared_w_gate_up=None, shared_w_down=None) -> moe_weights:
+                 s_down=None, shared_w_gate_up=None, shared_w_down=None, g_gate_up=None,
+                 g_down=None) -> moe_weights:
     return moe_weights(_ptr(router_w), _ptr(correction_bias), _ptr(w_gate_up), _ptr(s_gate_up),
-                       _ptr(w_down), _ptr(s_down), _ptr(shared_w_gate_up), _ptr(shared_w_down))
+                       _ptr(w_down), _ptr(s_down), _ptr(shared_w_gate_up), _ptr(shared_w_down),
+                       _ptr(g_gate_up), _ptr(g_down))
+
+
+def weight_format(w_gate_up, g_gate_up=None) -> int:
+    """The moe_weight_format of a layer's routed tensors: bf16 weights, or
+    uint8 codes -- NVFP4 when the per-expert fp32 tensor scales are given,
+    else W4A16."""
+    if g_gate_up is not None:
+        return MOE_W_NVFP4
+    return MOE_W_INT4_G128 if str(w_gate_up.dtype) == "torch.uint8" else MOE_W_BF16
 
 
 # ------------------------------------------------------- C entry points ----

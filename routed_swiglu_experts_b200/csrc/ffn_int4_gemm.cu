@@ -26,11 +26,22 @@
 // {0, 4, 1, 5, 2, 6, 3, 7} (how four LOP3s split a 32-bit code word); the
 // tokens are prepared in the same order, and the gate/up epilogue writes h
 // in it, so the K sum is unchanged.
+// NVFP4 experts (the module summary's routed NVFP4 MoE) run on the same
+// kernel with FP4 = true: the codes are FP4 E2M1 values packed the same way,
+// each 16 of K share one FP8 E4M3 scale, and each expert's weight tensor has
+// one fp32 scale.  The dequantisation warps form e2m1 * e4m3 in fp16 --
+// exact: at most 6 significant bits, magnitude 0 or within [2^-10, 2688] --
+// with the hardware e2m1 -> fp16 conversion, and the epilogues multiply the
+// fp32 accumulators by the tensor scale.  The activations stay 16-bit: the
+// pages state no activation quantisation, so the block-scaled fp4 x fp4 MMA
+// (which would quantise the tokens too) is not used.
 // Tiles are handed out from a queue in the workspace header as in the bf16
 // kernel.  Every mbarrier wait is bounded (MOE_ERR_DEVICE_TIMEOUT on expiry).
 #include <cstring>
 
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 
 #include "moe_internal.h"
 
@@ -64,7 +75,9 @@ struct alignas(64) Int4Params {
   CUtensorMap tma_q;          // codes: gate/up {K/2, 8, 2, N/8, G} box {128, 8, 2, 8, 1}; down {K/2, N, G} box {128, 128, 1}
   CUtensorMap tma_x;          // fp16 tokens {K, rows} box {64, 128}, 128-byte swizzle
   const int32_t* offsets;     // [groups + 1]
-  const __nv_bfloat16* scales;  // gate/up [G, 2N, K/128]; down [G, N, K/128]
+  const void* scales;         // int4: bf16 gate/up [G, 2N, K/128], down [G, N, K/128];
+                              // NVFP4: E4M3 bytes gate/up [G, 2N, K/16], down [G, N, K/16]
+  const float* tscale;        // NVFP4: fp32 tensor scale per expert (nullptr for int4)
   void* out;                  // gate/up: fp16 h [rows, N]; down: bf16 y [rows, N]
   const float* row_scale;     // down: per token row (or nullptr)
   int32_t groups;
@@ -154,6 +167,27 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
   return r;
 }
 
+// One word of FP4 E2M1 codes (k = 0..7 of an aligned 8, low nibble = even k)
+// -> four fp16x2 weights in the same {k0, k4}, {k1, k5}, {k2, k6}, {k3, k7}
+// order as dequant_word, each times its block's E4M3 scale s2 = (s, s).  The
+// conversion gives (k_even, k_odd) per byte; byte permutes regroup them.
+// Every product is exact in fp16 (see the file comment).
+__device__ __forceinline__ uint4 dequant_word_fp4(uint32_t w, uint32_t s2) {
+  uint32_t p[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const __half2_raw h =
+        __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>((w >> (8 * b)) & 0xFFu), __NV_E2M1);
+    p[b] = static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+  }
+  uint4 r;
+  r.x = hmul2_u(__byte_perm(p[0], p[2], 0x5410), s2);  // k0, k4
+  r.y = hmul2_u(__byte_perm(p[0], p[2], 0x7632), s2);  // k1, k5
+  r.z = hmul2_u(__byte_perm(p[1], p[3], 0x5410), s2);  // k2, k6
+  r.w = hmul2_u(__byte_perm(p[1], p[3], 0x7632), s2);  // k3, k7
+  return r;
+}
+
 // Reader side of the tile-id ring: wait until slot q holds the next id (it
 // may have been stored by the other CTA of the pair: cluster-scope acquire).
 __device__ __forceinline__ bool wait_tile(Ctl& c, int q, uint32_t qph, volatile int32_t* abort, uint64_t limit_ns,
@@ -176,7 +210,7 @@ __device__ __forceinline__ int slot_of(int f) {
   return (f & ~7) | ((j & 3) * 2 + (j >> 2));
 }
 
-template <Kind KIND>
+template <Kind KIND, bool FP4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     ffn_int4_pair_kernel(const __grid_constant__ Int4Params P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -472,26 +506,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       next_slot(q, qph);
       if (t < 0) break;
       const Tile ti = decode(P, c, t);
-      // this row's scales (nullptr: past the end of the matrix, codes are zero-filled)
-      const __nv_bfloat16* sp = nullptr;
+      // this row of the scale arrays (-1: past the end of the matrix, codes are zero-filled)
+      int64_t srow = -1;
       if (KIND == Kind::GateUp) {
         const int f = ti.fidx * 128 + static_cast<int>(rank) * 64 + (i >> 4) * 8 + (i & 7);
         const int u = (i >> 3) & 1;
-        if (f < P.n_out)
-          sp = P.scales + (static_cast<size_t>(ti.g) * 2 * P.n_out + static_cast<size_t>(u) * P.n_out + f) * groups;
+        if (f < P.n_out) srow = (static_cast<int64_t>(ti.g) * 2 + u) * P.n_out + f;
       } else {
         const int n = ti.fidx * 256 + static_cast<int>(rank) * 128 + i;
-        if (n < P.n_out) sp = P.scales + (static_cast<size_t>(ti.g) * P.n_out + n) * groups;
+        if (n < P.n_out) srow = static_cast<int64_t>(ti.g) * P.n_out + n;
       }
+      const __nv_bfloat16* sp =
+          (!FP4 && srow >= 0) ? static_cast<const __nv_bfloat16*>(P.scales) + srow * groups : nullptr;
+      // NVFP4: this thread's two E4M3 block scales per K step (blocks 4 kb + 2 half, + 1),
+      // loaded one step ahead
+      const unsigned short* sp8 =
+          (FP4 && srow >= 0)
+              ? reinterpret_cast<const unsigned short*>(static_cast<const unsigned char*>(P.scales) +
+                                                        srow * (P.K / 16)) + half
+              : nullptr;
+      unsigned short s8_next = (sp8 != nullptr && P.k_blocks > 0) ? __ldg(sp8) : 0;
       uint4 sv = make_uint4(0, 0, 0, 0), sn = sv;
-      if (batch8 && sp != nullptr) {
+      if (!FP4 && batch8 && sp != nullptr) {
         sv = __ldg(reinterpret_cast<const uint4*>(sp));
         if (groups > 8) sn = __ldg(reinterpret_cast<const uint4*>(sp + 8));
       }
       bool ok = true;
       for (int kb = 0; kb < P.k_blocks; ++kb) {
         const int gq = kb >> 1;
-        if (batch8 && (kb & 15) == 0 && kb > 0) {  // next batch of 8 groups
+        if (!FP4 && batch8 && (kb & 15) == 0 && kb > 0) {  // next batch of 8 groups
           sv = sn;
           if (sp != nullptr && gq + 8 < groups) sn = __ldg(reinterpret_cast<const uint4*>(sp + gq + 8));
         }
@@ -509,6 +552,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const __half2 s16h = __floats2half2_rn(sf * 0.0625f, sf * 0.0625f);
         const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&s2h);
         const uint32_t s2_16 = *reinterpret_cast<const uint32_t*>(&s16h);
+        uint32_t s2a = 0, s2b = 0;  // NVFP4: (s, s) of the thread's first and second 16 of K
+        if (FP4) {
+          const unsigned short s8 = s8_next;
+          if (sp8 != nullptr && kb + 1 < P.k_blocks) s8_next = __ldg(sp8 + 2 * (kb + 1));
+          const __half2_raw sh = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(s8), __NV_E4M3);
+          const uint32_t both = static_cast<uint32_t>(sh.x) | (static_cast<uint32_t>(sh.y) << 16);
+          s2a = __byte_perm(both, 0, 0x1010);
+          s2b = __byte_perm(both, 0, 0x3232);
+        }
         // codes landed (first K step of a copy), and the MMAs have released this A stage
         const int sub = kb % CKB;
         const bool got = (sub != 0 || mbar_wait_bounded(&c.code_full[cs], cphase, abort_flag, P.wait_ns)) &&
@@ -534,7 +586,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const int j = half * 4 + jj;  // 16-byte chunk of the 128-byte row
-          *reinterpret_cast<uint4*>(dst + ((j ^ (i & 7)) << 4)) = dequant_word(qw[jj], s2, s2_16);
+          *reinterpret_cast<uint4*>(dst + ((j ^ (i & 7)) << 4)) =
+              FP4 ? dequant_word_fp4(qw[jj], jj < 2 ? s2a : s2b) : dequant_word(qw[jj], s2, s2_16);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -580,6 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // the gate and the up value of one feature (as in the bf16 kernel)
         const int f0 = ti.fidx * 128 + static_cast<int>(rank) * 64;
         const float L = P.limit;
+        const float ts = FP4 ? __ldg(P.tscale + ti.g) : 1.f;
         unsigned char* hb = reinterpret_cast<unsigned char*>(c.obuf);
         __half* outh = static_cast<__half*>(P.out);
 #pragma unroll 1
@@ -598,8 +652,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 const int tok = 8 * q + 2 * (lane & 3) + e;
-                const float gv = fminf(__uint_as_float(v[h][4 * q + e]), L);
-                const float uv = fminf(fmaxf(__uint_as_float(v[h][4 * q + 2 + e]), -L), L);
+                const float graw = __uint_as_float(v[h][4 * q + e]);
+                const float uraw = __uint_as_float(v[h][4 * q + 2 + e]);
+                const float gv = fminf(FP4 ? graw * ts : graw, L);
+                const float uv = fminf(fmaxf(FP4 ? uraw * ts : uraw, -L), L);
                 const float hv = __bfloat162float(__float2bfloat16_rn(__fdividef(gv, 1.f + __expf(-gv)) * uv));
                 *reinterpret_cast<__half*>(hb + tok * HPITCH + fl * 2) = __float2half_rn(hv);
               }
@@ -622,6 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int nl = warp * 32 + lane;
         const int n0 = ti.fidx * 256 + static_cast<int>(rank) * 128;
         const float* rs = P.row_scale;
+        const float ts = FP4 ? __ldg(P.tscale + ti.g) : 1.f;
 #pragma unroll 1
         for (int ch = 0; ch < nch; ++ch) {
           uint32_t v[32];
@@ -629,7 +686,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           tmem_ld32(tbase + ch * 32, v);
           tmem_ld_wait();
           const int mycol = ch * 32 + lane;
-          const float my_sc = (rs != nullptr && mycol < ti.ntok) ? rs[ti.row0 + mycol] : 1.f;
+          const float rsv = (rs != nullptr && mycol < ti.ntok) ? rs[ti.row0 + mycol] : 1.f;
+          const float my_sc = FP4 ? rsv * ts : rsv;
           named_barrier_sync(1, 128);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -718,7 +776,7 @@ bool encode_tokens16(CUtensorMap* m, const void* base, int rows, int K) {
   return encode_tma(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <Kind KIND>
+template <Kind KIND, bool FP4>
 int resident_pairs_int4() {
   static int cached[64];
   static bool known[64];
@@ -731,7 +789,7 @@ int resident_pairs_int4() {
     lc.blockDim = dim3(THREADS);
     lc.dynamicSmemBytes = kSmem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, ffn_int4_pair_kernel<KIND>, &lc) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_int4_pair_kernel<KIND, FP4>, &lc) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
@@ -741,10 +799,11 @@ int resident_pairs_int4() {
   return cached[dev];
 }
 
-template <Kind KIND>
+template <Kind KIND, bool FP4>
 cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offsets, int groups, const void* q,
-                             const void* scales, int N, int K, void* out, const float* row_scale, float limit,
-                             int32_t* err, int32_t* queue, int num_sms, cudaStream_t stream) {
+                             const void* scales, const float* tscale, int N, int K, void* out,
+                             const float* row_scale, float limit, int32_t* err, int32_t* queue, int num_sms,
+                             cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   if (queue == nullptr) return cudaErrorInvalidValue;
   Int4Params P;
@@ -754,7 +813,8 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
                                         : encode_codes_d(&P.tma_q, q, groups, N, K);
   if (!okq) return cudaErrorInvalidValue;
   P.offsets = offsets;
-  P.scales = static_cast<const __nv_bfloat16*>(scales);
+  P.scales = scales;
+  P.tscale = tscale;
   P.out = out;
   P.row_scale = row_scale;
   P.groups = groups;
@@ -767,12 +827,13 @@ cudaError_t launch_int4_pair(const void* tokens16, int rows, const int32_t* offs
   P.err = err;
   P.queue = queue;
   P.wait_ns = kTimeoutNs;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<KIND>), static_cast<int>(kSmem));
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<KIND, FP4>), static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
   int grid = std::max(2, num_sms / 2 * 2);
-  const int pairs = resident_pairs_int4<KIND>();
+  const int pairs = resident_pairs_int4<KIND, FP4>();
   if (pairs > 0) grid = std::min(grid, 2 * pairs);
-  return launch_kernel(ffn_int4_pair_kernel<KIND>, dim3(grid), dim3(THREADS), kSmem, stream, P);
+  return launch_kernel(ffn_int4_pair_kernel<KIND, FP4>, dim3(grid), dim3(THREADS), kSmem, stream, P);
 }
 
 }  // namespace
@@ -799,7 +860,7 @@ cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32
   if (!encode_tokens16(&P.tma_x, tokens16, 16, 256) || !encode_codes_gu(&P.tma_q, q, 1, 64, 256))
     return cudaErrorInvalidValue;
   P.offsets = offsets;
-  P.scales = static_cast<const __nv_bfloat16*>(scales);
+  P.scales = scales;
   P.out = h16;
   P.groups = 1;
   P.rows = 16;
@@ -812,9 +873,10 @@ cudaError_t launch_int4_pair_timeout_selftest(void* scratch, int32_t* err, int32
   P.queue = queue;
   P.wait_ns = 20000000ull;
   P.test_withhold = 1;
-  e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<Kind::GateUp>), static_cast<int>(kSmem));
+  e = ensure_smem_attr(reinterpret_cast<const void*>(ffn_int4_pair_kernel<Kind::GateUp, false>),
+                       static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
-  ffn_int4_pair_kernel<Kind::GateUp><<<2, THREADS, kSmem, stream>>>(P);
+  ffn_int4_pair_kernel<Kind::GateUp, false><<<2, THREADS, kSmem, stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -830,11 +892,18 @@ cudaError_t launch_int4_ffn_prefill(const moe_config& cfg, const moe_weights& w,
                                         static_cast<const __nv_bfloat16*>(x_rows), H / 8, gather_src, cfg.top_k,
                                         static_cast<uint4*>(tokens16));
   if (e != cudaSuccess) return e;
-  e = launch_int4_pair<Kind::GateUp>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, I, H, h16, nullptr,
-                                     cfg.swiglu_limit, err, queues, num_sms, stream);
+  if (cfg.expert_format == MOE_W_NVFP4) {
+    e = launch_int4_pair<Kind::GateUp, true>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, w.g_gate_up, I, H,
+                                             h16, nullptr, cfg.swiglu_limit, err, queues, num_sms, stream);
+    if (e != cudaSuccess) return e;
+    return launch_int4_pair<Kind::Down, true>(h16, rows, offsets, E, w.w_down, w.s_down, w.g_down, H, I, y_perm,
+                                              w_perm, 0.f, err, queues + 2, num_sms, stream);
+  }
+  e = launch_int4_pair<Kind::GateUp, false>(tokens16, rows, offsets, E, w.w_gate_up, w.s_gate_up, nullptr, I, H, h16,
+                                            nullptr, cfg.swiglu_limit, err, queues, num_sms, stream);
   if (e != cudaSuccess) return e;
-  return launch_int4_pair<Kind::Down>(h16, rows, offsets, E, w.w_down, w.s_down, H, I, y_perm, w_perm, 0.f, err,
-                                      queues + 2, num_sms, stream);
+  return launch_int4_pair<Kind::Down, false>(h16, rows, offsets, E, w.w_down, w.s_down, nullptr, H, I, y_perm, w_perm,
+                                             0.f, err, queues + 2, num_sms, stream);
 }
 
 }  // namespace moe

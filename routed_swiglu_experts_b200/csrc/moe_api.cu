@@ -56,14 +56,22 @@ int32_t* tile_queue(void* ws, TileQueueSlot slot) { return reinterpret_cast<WsHe
 int32_t* perm_ticket(void* ws) { return &reinterpret_cast<WsHeader*>(ws)->perm_done; }
 
 bool is_int4(const moe_config& cfg) { return cfg.expert_format == MOE_W_INT4_G128; }
+bool is_nvfp4(const moe_config& cfg) { return cfg.expert_format == MOE_W_NVFP4; }
+// both 4-bit formats: fp16 activations, the 4-bit kernels gather the routed rows
+bool is_4bit(const moe_config& cfg) { return is_int4(cfg) || is_nvfp4(cfg); }
 
 moe_status check_expert_weights(const moe_config& cfg, const moe_weights* w) {
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   if (w->w_gate_up == nullptr || w->w_down == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->w_gate_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
-  if (is_int4(cfg)) {
+  if (is_4bit(cfg)) {
     if (w->s_gate_up == nullptr || w->s_down == nullptr) return MOE_ERR_INVALID_ARG;
     if (!aligned16(w->s_gate_up) || !aligned16(w->s_down)) return MOE_ERR_INVALID_ARG;
+  }
+  if (is_nvfp4(cfg)) {
+    if (w->g_gate_up == nullptr || w->g_down == nullptr) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(w->g_gate_up) & 3u) != 0 || (reinterpret_cast<uintptr_t>(w->g_down) & 3u) != 0)
+      return MOE_ERR_INVALID_ARG;
   }
   return MOE_OK;
 }
@@ -101,7 +109,8 @@ moe_status check_router_weights(const moe_weights* w) {
 // computes (0 allowed: shared expert only), `offsets` their [E + 1] row
 // offsets (absolute permuted rows), and w's routed weights hold exactly those
 // experts; e_total is the router's expert count (the int4 path picks its
-// kernel by the average routed rows per expert, R / e_total).
+// kernel by the average routed rows per expert, R / e_total; NVFP4 experts
+// always take the grouped tensor-core kernel).
 moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_rows, const int32_t* gather_src,
                    const int32_t* offsets, const float* w_perm, int32_t T, void* y_perm, const void* x_shared,
                    void* shared_out, void* ws, const WsLayout& L, cudaStream_t stream, int e_total) {
@@ -119,7 +128,7 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_ro
   // few tokens: the shared expert streams its weights with the split-K
   // kernels -- or, beside the int4 GEMVs, inside their launches; otherwise it
   // is one more problem of the tcgen05 launches
-  const bool prefill_path = is_int4(cfg) && int4_prefill_preferred(R, e_total);
+  const bool prefill_path = is_nvfp4(cfg) || (is_int4(cfg) && int4_prefill_preferred(R, e_total));
   const bool gemv_path = is_int4(cfg) && !prefill_path;
   const bool shared_in_gemv = with_shared && gemv_path && w4a16_shared_fusable(T, Is);
   const bool shared_small = with_shared && !shared_in_gemv && dense_small_ok(T, H, Is);
@@ -132,7 +141,7 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_ro
   if (shared_small)
     MOE_CUDA_TRY(launch_dense_small_ffn(x_shared, T, H, Is, w.shared_w_gate_up, w.shared_w_down, cfg.swiglu_limit,
                                         at<float>(ws, L.small_part), hs, shared_out, err, sms, stream));
-  if (!is_int4(cfg)) {
+  if (!is_4bit(cfg)) {
     FfnProblem r_gu{x_rows, R, offsets, E, w.w_gate_up, I, H, h, nullptr, gather_src, cfg.top_k, T};
     FfnProblem r_d{h, R, offsets, E, w.w_down, H, I, y_perm, w_perm};
     MOE_CUDA_TRY(launch_gemm_gateup(routed ? &r_gu : nullptr, shared_tc ? &s_gu : nullptr, cfg.swiglu_limit, err, qgu,
@@ -165,15 +174,16 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_ro
 // copies them into the workspace's x_perm and the tensor-core kernel loads
 // contiguous token boxes (its per-row gather4 form, moe_grouped_swiglu_ffn_gather,
 // takes about twice as long: one TMA copy per four 128-byte rows is
-// latency-bound).  int4 experts: the permute writes the maps only and the
-// activation conversion that every int4 kernel runs first gathers the rows.
+// latency-bound).  int4 and NVFP4 experts: the permute writes the maps only
+// and the activation conversion that every 4-bit kernel runs first gathers
+// the rows.
 struct Rows {
   void* x_perm;                 // permute output, or nullptr (maps only)
   const void* x_rows;           // what run_ffn reads
   const int32_t* gather_src;    // nullptr, or the slot map of a gathered read
 };
 Rows routed_rows(const moe_config& cfg, void* ws, const WsLayout& L, const void* x, const int32_t* src) {
-  if (is_int4(cfg)) return Rows{nullptr, x, src};
+  if (is_4bit(cfg)) return Rows{nullptr, x, src};
   void* xp = at<void>(ws, L.x_perm);
   return Rows{xp, xp, nullptr};
 }
@@ -220,18 +230,19 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.block_base = take(static_cast<size_t>(perm_blocks(static_cast<int>(R))) * E * sizeof(int32_t));
   L.local_rank = take(R * sizeof(int32_t));
   const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
+  const bool four = int4 || cfg.expert_format == MOE_W_NVFP4;
   // bf16 experts: the forward gathers the routed rows into x_perm (tiled TMA
-  // copies then feed the tensor cores); int4 experts gather while converting
-  L.x_perm = take(int4 ? 0 : R * H * 2);
-  // bf16 h, or the int4 kernels' h: fp16 [R, I] (grouped GEMM) or fp32 gate/up
-  // [R, 2I] (GEMVs, taken only below kInt4PrefillRowsPerExpert rows per expert)
+  // copies then feed the tensor cores); 4-bit experts gather while converting
+  L.x_perm = take(four ? 0 : R * H * 2);
+  // bf16 h, the 4-bit grouped GEMMs' fp16 h [R, I], or the int4 GEMVs' fp32
+  // gate/up [R, 2I] (taken only below kInt4PrefillRowsPerExpert rows per expert)
   const size_t r_gemv = std::min(R, static_cast<size_t>(kInt4PrefillRowsPerExpert) * E);
   L.h = take(int4 ? std::max(R * I * 2, r_gemv * 2 * I * 4) : R * I * 2);
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
   L.shared_out = take(T * H * 2);
   const size_t kmax = std::max(H, I);
-  L.act16 = take(int4 ? R * kmax * 2 : 0);
+  L.act16 = take(four ? R * kmax * 2 : 0);
   L.small_part = take(Is > 0 ? dense_small_part_floats(static_cast<int>(H), static_cast<int>(Is)) * sizeof(float) : 0);
   L.total = off;
   return L;
@@ -268,12 +279,12 @@ moe_status moe_config_validate(const moe_config* cfg) {
   if (std::isnan(c.swiglu_limit) || !(c.swiglu_limit > 0.f)) return MOE_ERR_INVALID_ARG;
   if (!std::isfinite(c.routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
   if (c.renormalize != 0 && c.renormalize != 1) return MOE_ERR_INVALID_ARG;
-  if (c.expert_format != MOE_W_BF16 && c.expert_format != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
-  if (c.expert_format == MOE_W_INT4_G128 && (c.hidden % 128 != 0 || c.expert_inter % 128 != 0))
-    return MOE_ERR_UNSUPPORTED;
-  // the int4 paths feed h to fp16 tensor-core operands: |h| <= L^2 must stay finite in fp16
-  if (c.expert_format == MOE_W_INT4_G128 && !(c.swiglu_limit <= MOE_INT4_MAX_SWIGLU_LIMIT))
-    return MOE_ERR_UNSUPPORTED;
+  if (c.expert_format != MOE_W_BF16 && c.expert_format != MOE_W_INT4_G128 && c.expert_format != MOE_W_NVFP4)
+    return MOE_ERR_INVALID_ARG;
+  const bool four = c.expert_format != MOE_W_BF16;
+  if (four && (c.hidden % 128 != 0 || c.expert_inter % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  // the 4-bit paths feed h to fp16 tensor-core operands: |h| <= L^2 must stay finite in fp16
+  if (four && !(c.swiglu_limit <= MOE_INT4_MAX_SWIGLU_LIMIT)) return MOE_ERR_UNSUPPORTED;
   // TMA strides and boxes: rows of up to 2^31 bytes
   if (static_cast<int64_t>(c.hidden) * 2 >= (int64_t(1) << 31) ||
       static_cast<int64_t>(c.expert_inter) * 2 >= (int64_t(1) << 31))

@@ -127,11 +127,12 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
                               int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
                               int T, void* h_shared, void* shared_out, cudaStream_t stream);
 
-// W4A16 grouped GEMMs for many tokens per expert: int4 codes dequantised to
-// fp16 in shared memory and fed to the CTA-pair tensor-core pipeline.
+// 4-bit grouped GEMMs: int4 (W4A16, for many tokens per expert: at least
+// kInt4PrefillRowsPerExpert routed rows per expert on average) or NVFP4 (at
+// every token count) codes dequantised to fp16 in shared memory and fed to
+// the CTA-pair tensor-core pipeline; cfg.expert_format picks the decoder.
 // tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16; queues:
 // four tile-queue words in the workspace header (gate/up, then down).
-// (at least kInt4PrefillRowsPerExpert routed rows per expert on average)
 constexpr int kInt4PrefillRowsPerExpert = 32;
 bool int4_prefill_preferred(int rows, int E);
 // x_rows / gather_src as for launch_w4a16_gateup.

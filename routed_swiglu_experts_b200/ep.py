@@ -47,7 +47,8 @@ def shared_slices(shared_inter: int, world: int, unit: int = 8) -> List[Tuple[in
 
 
 def local_tensors(rank: int, world: int, num_experts: int, shared_inter: int, *, w_gate_up, w_down,
-                  s_gate_up=None, s_down=None, shared_w_gate_up=None, shared_w_down=None) -> dict:
+                  s_gate_up=None, s_down=None, shared_w_gate_up=None, shared_w_down=None,
+                  g_gate_up=None, g_down=None) -> dict:
     """The weight tensors rank `rank` holds: its experts' rows of the routed
     tensors ([E, ...] -> [E_local, ...]) and its slice of the shared expert
     (gate rows [s0, s1) then up rows [I_s + s0, I_s + s1) of the fused gate/up
@@ -61,6 +62,8 @@ def local_tensors(rank: int, world: int, num_experts: int, shared_inter: int, *,
         "w_down": w_down[b:e].contiguous(),
         "s_gate_up": None if s_gate_up is None else s_gate_up[b:e].contiguous(),
         "s_down": None if s_down is None else s_down[b:e].contiguous(),
+        "g_gate_up": None if g_gate_up is None else g_gate_up[b:e].contiguous(),
+        "g_down": None if g_down is None else g_down[b:e].contiguous(),
         "shared_w_gate_up": None,
         "shared_w_down": None,
         "expert_range": (b, e),
@@ -82,14 +85,14 @@ class ExpertParallelLayer:
     def __init__(self, *, hidden, num_experts, top_k, expert_inter, shared_inter, swiglu_limit,
                  routed_scaling_factor, renormalize, router_w, correction_bias, w_gate_up, w_down,
                  s_gate_up=None, s_down=None, shared_w_gate_up=None, shared_w_down=None,
-                 rank: int = 0, world: int = 1, max_tokens: int = 0, group=None):
-        import torch
+                 g_gate_up=None, g_down=None, rank: int = 0, world: int = 1, max_tokens: int = 0,
+                 group=None):
         loc = local_tensors(rank, world, num_experts, shared_inter, w_gate_up=w_gate_up, w_down=w_down,
                             s_gate_up=s_gate_up, s_down=s_down, shared_w_gate_up=shared_w_gate_up,
-                            shared_w_down=shared_w_down)
+                            shared_w_down=shared_w_down, g_gate_up=g_gate_up, g_down=g_down)
         self.expert_range = loc["expert_range"]
         s0, s1 = loc["shared_slice"]
-        fmt = _abi.MOE_W_INT4_G128 if w_gate_up.dtype == torch.uint8 else _abi.MOE_W_BF16
+        fmt = _abi.weight_format(w_gate_up, g_gate_up)
         self.cfg = _abi.make_config(hidden, num_experts, top_k, expert_inter, s1 - s0, swiglu_limit,
                                     routed_scaling_factor, renormalize, fmt)
         st = _abi.moe_config_validate(self.cfg)
@@ -99,6 +102,7 @@ class ExpertParallelLayer:
         self.tensors = dict(router_w=router_w, correction_bias=correction_bias,
                             w_gate_up=None if empty else loc["w_gate_up"], w_down=None if empty else loc["w_down"],
                             s_gate_up=None if empty else loc["s_gate_up"], s_down=None if empty else loc["s_down"],
+                            g_gate_up=None if empty else loc["g_gate_up"], g_down=None if empty else loc["g_down"],
                             shared_w_gate_up=loc["shared_w_gate_up"], shared_w_down=loc["shared_w_down"])
         self.w = _abi.make_weights(**self.tensors)
         self.device = router_w.device

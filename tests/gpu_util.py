@@ -12,7 +12,8 @@ import torch
 import routed_swiglu_experts_b200 as rse
 
 # Layer-output tolerance: max|gpu - oracle| <= TOL * max|oracle| over the
-# compared rows (bf16 weights), doubled for W4A16 weights.
+# compared rows (bf16 weights), doubled for 4-bit (W4A16, NVFP4) weights:
+# their kernels run on fp16 activations.
 TOL_BF16 = 2e-2
 TOL_W4A16 = 4e-2
 # Near-tie exemption on the oracle's k-th vs (k+1)-th biased-score gap.
@@ -35,6 +36,7 @@ def gpu_layer(inp, max_tokens: Optional[int] = None) -> rse.MoELayer:
         router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias), w_gate_up=mv(inp.w_gate_up),
         w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up), s_down=mv(inp.s_down),
         shared_w_gate_up=mv(inp.shared_w_gate_up), shared_w_down=mv(inp.shared_w_down),
+        g_gate_up=mv(inp.g_gate_up), g_down=mv(inp.g_down),
         max_tokens=max_tokens if max_tokens is not None else inp.x.shape[0])
 
 
@@ -119,4 +121,4 @@ def check_ids(gpu_ids: torch.Tensor, sel, tie_gap: float = TIE_GAP):
 
 
 def tol_for(cfg) -> float:
-    return TOL_W4A16 if cfg.w4a16 else TOL_BF16
+    return TOL_W4A16 if (cfg.w4a16 or cfg.nvfp4) else TOL_BF16

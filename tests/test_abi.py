@@ -84,9 +84,16 @@ def mid_cfg(**kw):
     ({"expert_format": _abi.MOE_W_INT4_G128, "swiglu_limit": 256.0}, _abi.MOE_ERR_UNSUPPORTED),
     ({"expert_format": _abi.MOE_W_INT4_G128, "swiglu_limit": 255.0}, _abi.MOE_OK),
     ({"swiglu_limit": 1e30}, _abi.MOE_OK),                # bf16 experts: no such bound
+    # NVFP4 experts: the same multiples of 128 and the same fp16 bound on h
+    ({"expert_format": _abi.MOE_W_NVFP4}, _abi.MOE_OK),
+    ({"expert_format": _abi.MOE_W_NVFP4, "expert_inter": 1416}, _abi.MOE_ERR_UNSUPPORTED),
+    ({"expert_format": _abi.MOE_W_NVFP4, "hidden": 2056}, _abi.MOE_ERR_UNSUPPORTED),
+    ({"expert_format": _abi.MOE_W_NVFP4, "swiglu_limit": 256.0}, _abi.MOE_ERR_UNSUPPORTED),
+    ({"expert_format": _abi.MOE_W_NVFP4, "swiglu_limit": 255.0}, _abi.MOE_OK),
+    ({"expert_format": 3}, _abi.MOE_ERR_INVALID_ARG),
 ])
 def test_config_validation(lib, kw, status):
-    if kw.get("expert_format") == _abi.MOE_W_INT4_G128 and "expert_inter" not in kw:
+    if kw.get("expert_format") in (_abi.MOE_W_INT4_G128, _abi.MOE_W_NVFP4) and "expert_inter" not in kw:
         kw = dict(kw, expert_inter=1536)
     assert _abi.moe_config_validate(mid_cfg(**kw)) == status
 
@@ -103,6 +110,13 @@ def test_workspace_size(lib):
     R4, I4 = 4096 * 6, 2048
     bf16_like = R4 * H * 2 + R4 * 2 * I4 * 4 + R4 * H * 2 + R4 * max(H, I4) * 2  # with an x_perm region
     assert _abi.moe_workspace_size(c4, 4096) < bf16_like + (64 << 20)
+    # NVFP4 experts: no x_perm region and no fp32 GEMV scratch (the grouped
+    # GEMM's fp16 h only): never more than the int4 layer of the same shape,
+    # and less at few tokens, where the int4 layer runs its GEMVs
+    cf = mid_cfg(expert_format=_abi.MOE_W_NVFP4, expert_inter=2048, hidden=2048)
+    for T in (1, 32, 4096):
+        assert _abi.moe_workspace_size(cf, T) <= _abi.moe_workspace_size(c4, T)
+    assert _abi.moe_workspace_size(cf, 1) < _abi.moe_workspace_size(c4, 1)
     with pytest.raises(rse.MoEError):
         _abi.moe_workspace_size(cfg, -1)
 
@@ -143,6 +157,17 @@ def test_forward_argument_checks(lib):
     c4 = mid_cfg(expert_format=_abi.MOE_W_INT4_G128, expert_inter=2048)
     assert _call_forward(lib, c4, _fake_weights()) == _abi.MOE_ERR_INVALID_ARG
     assert _call_forward(lib, c4, _fake_weights(s_gate_up=FAKE, s_down=FAKE), T=0) == _abi.MOE_OK
+    # NVFP4 experts need their block scales and their fp32 tensor scales (4-byte aligned)
+    cf = mid_cfg(expert_format=_abi.MOE_W_NVFP4, expert_inter=2048)
+    scaled = dict(s_gate_up=FAKE, s_down=FAKE)
+    assert _call_forward(lib, cf, _fake_weights(**scaled)) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_forward(lib, cf, _fake_weights(g_gate_up=FAKE, g_down=FAKE)) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_forward(lib, cf, _fake_weights(**scaled, g_gate_up=FAKE)) == _abi.MOE_ERR_INVALID_ARG
+    assert _call_forward(lib, cf, _fake_weights(**scaled, g_gate_up=FAKE, g_down=FAKE + 2)) == \
+        _abi.MOE_ERR_INVALID_ARG
+    assert _call_forward(lib, cf, _fake_weights(**scaled, g_gate_up=FAKE + 4, g_down=FAKE + 8), T=0) == _abi.MOE_OK
+    # the tensor scales are ignored for the other formats
+    assert _call_forward(lib, c4, _fake_weights(s_gate_up=FAKE, s_down=FAKE, g_down=FAKE + 2), T=0) == _abi.MOE_OK
     # bad configuration is reported first
     assert _call_forward(lib, mid_cfg(top_k=17), w) == _abi.MOE_ERR_UNSUPPORTED
 

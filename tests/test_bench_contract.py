@@ -37,6 +37,8 @@ def test_gemm_flops_of_the_mid_layer():
     # ... + token prep + dequantising gate/up and down + bf16 shared gate/up
     # and down launches
     ("prefill_w4a16", 11),
+    # NVFP4 experts take the same grouped kernels at every token count
+    ("prefill_nvfp4", 11),
 ])
 def test_launches_per_step_match_the_launch_lists(name, expected):
     assert bench.launches_per_step(CONFIGS[name]) == expected

@@ -31,11 +31,16 @@ CASES = {
                                  w4a16=True),
     # W4A16 grouped prefill GEMM
     "ep_w4a16_prefill": LayerConfig("ep_w4a16_prefill", T=300, H=256, E=4, k=2, I=256, I_s=128, w4a16=True),
+    # NVFP4 grouped GEMM (tensor scales sliced with the experts); shared slice on
+    # the tcgen05 launches, then on the split-K path
+    "ep_nvfp4": LayerConfig("ep_nvfp4", T=300, H=256, E=4, k=2, I=256, I_s=128, nvfp4=True),
+    "ep_nvfp4_few": LayerConfig("ep_nvfp4_few", T=20, H=256, E=6, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
+                                nvfp4=True),
     # more ranks than experts: the last rank has no expert, only a shared slice
     "ep_sparse": LayerConfig("ep_sparse", T=150, H=128, E=3, k=2, I=64, I_s=32),
 }
 WORLDS = {"ep_bf16": [1, 2, 3, 8], "ep_bf16_few": [2], "ep_w4a16_gemv": [2], "ep_w4a16_prefill": [2],
-          "ep_sparse": [4]}
+          "ep_nvfp4": [2], "ep_nvfp4_few": [3], "ep_sparse": [4]}
 
 
 @pytest.mark.parametrize("name,world", [(n, w) for n in CASES for w in WORLDS[n]])
@@ -55,6 +60,7 @@ def test_rank_partials_add_up_to_the_layer(name, world):
             router_w=mv(inp.router_w), correction_bias=mv(inp.correction_bias), w_gate_up=mv(inp.w_gate_up),
             w_down=mv(inp.w_down), s_gate_up=mv(inp.s_gate_up), s_down=mv(inp.s_down),
             shared_w_gate_up=mv(inp.shared_w_gate_up), shared_w_down=mv(inp.shared_w_down),
+            g_gate_up=mv(inp.g_gate_up), g_down=mv(inp.g_down),
             rank=r, world=world, max_tokens=cfg.T)
         ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
         part = layer.forward_partial(x, topk_ids=ids)

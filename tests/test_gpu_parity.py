@@ -16,7 +16,8 @@ printed line.
 Bars: expert ids and permutation indices bit-exact (router ids exempt only
 where the oracle's k-th vs (k+1)-th biased-score gap is below 1e-6; those
 are counted); routed weights within 1e-5 relative; outputs within
-max|gpu - oracle| <= 2e-2 * max|oracle| (bf16 weights) or 4e-2 (W4A16).
+max|gpu - oracle| <= 2e-2 * max|oracle| (bf16 weights) or 4e-2 (W4A16 and
+NVFP4 weights).
 """
 
 import math
@@ -66,6 +67,20 @@ EDGE = {
                                     swiglu_limit=255.0, x_scale=50.0, w4a16=True),
     "w4a16_prefill_wide_limit": LayerConfig("w4a16_prefill_wide_limit", T=300, H=256, E=4, k=2, I=256,
                                             I_s=128, swiglu_limit=255.0, x_scale=50.0, w4a16=True),
+    # NVFP4 experts (grouped tensor-core GEMM at every token count): few tokens
+    # (shared expert on the split-K path), several token and weight tiles with
+    # ragged tails (K = 384: the second code copy half past the row), many
+    # tiles per expert, the clamp, and the widest clamp with large activations
+    "nvfp4_small": LayerConfig("nvfp4_small", T=20, H=256, E=6, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
+                               bias_range=0.05, nvfp4=True),
+    "nvfp4_prefill": LayerConfig("nvfp4_prefill", T=700, H=512, E=8, k=2, I=384, I_s=256, alpha=2.5, renorm=True,
+                                 bias_range=0.05, nvfp4=True),
+    "nvfp4_wide": LayerConfig("nvfp4_wide", T=1500, H=1024, E=16, k=4, I=640, I_s=384, alpha=2.5, renorm=True,
+                              nvfp4=True),
+    "nvfp4_clamp": LayerConfig("nvfp4_clamp", T=300, H=256, E=4, k=2, I=256, I_s=128, swiglu_limit=0.5,
+                               nvfp4=True),
+    "nvfp4_wide_limit": LayerConfig("nvfp4_wide_limit", T=300, H=256, E=4, k=2, I=256, I_s=0,
+                                    swiglu_limit=255.0, x_scale=50.0, nvfp4=True),
     # enough tokens for the row-block top-k kernel: E not a multiple of 4
     # (scalar partial sums), and k >= 8 (17 kept values per thread)
     "rows_e5": LayerConfig("rows_e5", T=1300, H=128, E=5, k=3, I=64, I_s=32, alpha=1.5, renorm=True),
@@ -184,7 +199,7 @@ def test_forward_is_deterministic(small_inputs):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("name", ["ragged", "w4a16_prefill"])
+@pytest.mark.parametrize("name", ["ragged", "w4a16_prefill", "nvfp4_prefill"])
 def test_tile_queues_are_left_at_zero(small_inputs, name):
     """The persistent grouped GEMMs hand tiles out from counters in the
     workspace header; every launch must leave them at zero, so that the next
@@ -203,7 +218,7 @@ def test_tile_queues_are_left_at_zero(small_inputs, name):
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
-@pytest.mark.parametrize("name", ["ragged", "w4a16_small", "w4a16_prefill", "shared_small_t32"])
+@pytest.mark.parametrize("name", ["ragged", "w4a16_small", "w4a16_prefill", "nvfp4_small", "shared_small_t32"])
 def test_forward_replays_from_a_cuda_graph(small_inputs, name):
     """The forward enqueues only device work on the given stream (no host
     sync, no allocation): captured once into a CUDA graph, its replay gives
@@ -227,6 +242,33 @@ def test_forward_replays_from_a_cuda_graph(small_inputs, name):
     assert torch.equal(out, eager)
     assert layer.device_error() == 0
     del graph
+
+
+def test_nvfp4_every_scale_byte():
+    """The down weight's E4M3 block scales vary by output row and take every
+    finite E4M3 pattern (both signs, the subnormals, 448): output column n of
+    y_perm is one scale value times an unscaled sum, so each column is
+    compared with the oracle's on its own.  The E4M3 NaN patterns are left
+    out (they make NaN weights by definition)."""
+    cfg = LayerConfig("nvfp4_scales", T=300, H=256, E=2, k=1, I=128, I_s=0, nvfp4=True)
+    inp = moe_inputs.make_layer(cfg, seed=5)
+    finite = [b for b in range(256) if b not in (0x7F, 0xFF)] + [0x38, 0xB8]   # 256 rows
+    rows = torch.tensor(finite, dtype=torch.int64).to(torch.uint8)
+    inp.s_down = rows[None, :, None].expand(cfg.E, cfg.H, cfg.I // 16).contiguous()
+    layer = gpu_layer(inp)
+    st = run_stages(layer, inp.x.cuda())
+    res = oracle.moe_forward(inp, ids_override=st.ids.cpu().to(torch.int64))
+    y_ref = res.y_perm * st.w_perm.cpu().double()[:, None]
+    y = st.y_perm.cpu().double()
+    tol = tol_for(cfg)
+    for n in range(cfg.H):
+        m = float(y_ref[:, n].abs().max())
+        if m == 0.0:
+            assert bool((y[:, n] == 0).all()), f"scale byte {finite[n]:#04x}: column not zero"
+        else:
+            e = float((y[:, n] - y_ref[:, n]).abs().max()) / m
+            assert e <= tol, f"scale byte {finite[n]:#04x}: column error {e:.3e}"
+    assert layer.device_error() == 0
 
 
 @pytest.mark.parametrize("name", ["tied_router", "tied_router_rows"])
