@@ -31,8 +31,8 @@
 // each 16 of K share one FP8 E4M3 scale, and each expert's weight tensor has
 // one fp32 scale.  The dequantisation warps form e2m1 * e4m3 in fp16 --
 // exact: at most 6 significant bits, magnitude 0 or within [2^-10, 2688] --
-// with the hardware e2m1 -> fp16 conversion, and the epilogues multiply the
-// fp32 accumulators by the tensor scale.  The activations stay 16-bit: the
+// with the sm_100a conversions cvt.rn.f16x2.e2m1x2 and .e4m3x2, and the
+// epilogues multiply the fp32 accumulators by the tensor scale.  The activations stay 16-bit: the
 // pages state no activation quantisation, so the block-scaled fp4 x fp4 MMA
 // (which would quantise the tokens too) is not used.
 // Tiles are handed out from a queue in the workspace header as in the bf16
@@ -40,8 +40,6 @@
 #include <cstring>
 
 #include <cuda_fp16.h>
-#include <cuda_fp4.h>
-#include <cuda_fp8.h>
 
 #include "moe_internal.h"
 
@@ -170,21 +168,34 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
 // One word of FP4 E2M1 codes (k = 0..7 of an aligned 8, low nibble = even k)
 // -> four fp16x2 weights in the same {k0, k4}, {k1, k5}, {k2, k6}, {k3, k7}
 // order as dequant_word, each times its block's E4M3 scale s2 = (s, s).  The
-// conversion gives (k_even, k_odd) per byte; byte permutes regroup them.
-// Every product is exact in fp16 (see the file comment).
+// nibbles are first regrouped into the bytes k0|k4<<4, k2|k6<<4 (lo) and
+// k1|k5<<4, k3|k7<<4 (hi), so that each conversion (one E2M1 byte -> an
+// fp16 pair, low nibble in the low half) yields a finished pair.  Every
+// product is exact in fp16 (see the file comment).
 __device__ __forceinline__ uint4 dequant_word_fp4(uint32_t w, uint32_t s2) {
-  uint32_t p[4];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const __half2_raw h =
-        __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>((w >> (8 * b)) & 0xFFu), __NV_E2M1);
-    p[b] = static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-  }
+  const uint32_t lo = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
+  const uint32_t hi = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
   uint4 r;
-  r.x = hmul2_u(__byte_perm(p[0], p[2], 0x5410), s2);  // k0, k4
-  r.y = hmul2_u(__byte_perm(p[0], p[2], 0x7632), s2);  // k1, k5
-  r.z = hmul2_u(__byte_perm(p[1], p[3], 0x5410), s2);  // k2, k6
-  r.w = hmul2_u(__byte_perm(p[1], p[3], 0x7632), s2);  // k3, k7
+  asm("{\n\t.reg .b8 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+      "mov.b32 {a0, a1, a2, a3}, %4;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %5;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, a0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, a1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b1;\n\t}"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "r"(lo), "r"(hi));
+  r.x = hmul2_u(r.x, s2);  // k0, k4
+  r.y = hmul2_u(r.y, s2);  // k1, k5
+  r.z = hmul2_u(r.z, s2);  // k2, k6
+  r.w = hmul2_u(r.w, s2);  // k3, k7
+  return r;
+}
+
+// Two E4M3 scale bytes (low byte -> low half) to an fp16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(unsigned short v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
 }
 
@@ -556,8 +567,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (FP4) {
           const unsigned short s8 = s8_next;
           if (sp8 != nullptr && kb + 1 < P.k_blocks) s8_next = __ldg(sp8 + 2 * (kb + 1));
-          const __half2_raw sh = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(s8), __NV_E4M3);
-          const uint32_t both = static_cast<uint32_t>(sh.x) | (static_cast<uint32_t>(sh.y) << 16);
+          const uint32_t both = e4m3x2_to_f16x2(s8);
           s2a = __byte_perm(both, 0, 0x1010);
           s2b = __byte_perm(both, 0, 0x3232);
         }
