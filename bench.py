@@ -225,11 +225,16 @@ def run_cpu_baseline(inp, min_seconds=10.0, max_passes=20, gpu_out=None, gpu_ids
 
 
 def w4a16_bytes(cfg, ids):
-    """HBM bytes the W4A16 expert FFN call must move: codes + scales of every
-    touched expert, the bf16 shared expert, and its activations (the T*k
+    """HBM bytes the 4-bit expert FFN call must move: codes + scales of every
+    touched expert (W4A16: bf16 per 128; NVFP4: one byte per 16 and two fp32
+    tensor scales), the bf16 shared expert, and its activations (the T*k
     gathered token rows and x read, y_perm and the shared output written)."""
     touched = int(len(set(ids.reshape(-1).tolist())))
-    per_expert = (2 * cfg.I * cfg.H // 2 + cfg.H * cfg.I // 2) + 2 * (2 * cfg.I * cfg.H // 128 + cfg.H * cfg.I // 128)
+    codes = 2 * cfg.I * cfg.H // 2 + cfg.H * cfg.I // 2
+    if cfg.nvfp4:
+        per_expert = codes + (2 * cfg.I * cfg.H // 16 + cfg.H * cfg.I // 16) + 2 * 4
+    else:
+        per_expert = codes + 2 * (2 * cfg.I * cfg.H // 128 + cfg.H * cfg.I // 128)
     shared = 2 * (2 * cfg.I_s * cfg.H + cfg.H * cfg.I_s)
     acts = 2 * cfg.T * cfg.H * (2 + 2 * cfg.k)
     return touched, touched * per_expert + shared + acts
@@ -243,9 +248,9 @@ def launches_per_step(cfg):
     FFN path and the shared expert's launches when it does not ride in the
     routed ones."""
     n = 6
-    # 4-bit codes dequantised in shared memory, tensor cores (NVFP4 always)
-    prefill = cfg.nvfp4 or (cfg.w4a16 and cfg.T * cfg.k >= 32 * cfg.E)
-    gemv = cfg.w4a16 and not prefill                      # int4 dequantised in registers
+    four = cfg.w4a16 or cfg.nvfp4
+    prefill = four and cfg.T * cfg.k >= 32 * cfg.E       # 4-bit codes dequantised in shared memory, tensor cores
+    gemv = four and not prefill                           # 4-bit codes dequantised in registers
     shared = 0
     if cfg.I_s > 0:
         if gemv and cfg.T <= 32:
@@ -559,11 +564,12 @@ def bench_ours(args, rank, world, local_rank):
     peaks = measured_peaks()
     routed_f, shared_f = gemm_flops(c)
     ffn_s = stage_ms["grouped_ffn"] / 1e3
-    if c.w4a16 and c.T * c.k < 32 * c.E:  # the GEMV path: HBM-bound
+    if (c.w4a16 or c.nvfp4) and c.T * c.k < 32 * c.E:  # the GEMV path: HBM-bound
         touched, nbytes = w4a16_bytes(c, ids.cpu())
         achieved = nbytes / ffn_s / 1e9
-        roof = {"kernel": "W4A16 expert FFN (register-dequant gate/up and down GEMV launches with their "
-                          "activation preps) + bf16 shared expert", "bound": "hbm", "achieved": achieved,
+        roof = {"kernel": ("NVFP4" if c.nvfp4 else "W4A16") + " expert FFN (register-dequant gate/up and down GEMV "
+                          "launches with their activation preps) + bf16 shared expert", "bound": "hbm",
+                "achieved": achieved,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                 "traffic": traffic_from_profile(f"grouped_ffn_{c.name}"),
                 "peak_source": f"{peaks['source']} HBM copy", "bytes_per_call": nbytes,

@@ -140,10 +140,10 @@ typedef struct moe_weights {
  * FP8 E4M3 of 8-bit Floating Point): byte q[n, c] holds the E2M1 codes of
  * k = 2c (low nibble) and k = 2c + 1 (high nibble);
  *   w[n, k] = e2m1(code) * e4m3(s[n, k / 16]) * g[e].
- * The grouped tensor-core GEMM forms e2m1 * e4m3 in fp16, which is exact for
- * every finite E4M3 scale (the E4M3 NaN patterns give NaN weights), and
- * multiplies the fp32 accumulators by g[e]; the activation limits of the
- * W4A16 range note above (fp16 x and h, swiglu_limit) hold as stated there. */
+ * Both NVFP4 kernels form e2m1 * e4m3 in fp16, which is exact for every
+ * finite E4M3 scale (the E4M3 NaN patterns give NaN weights), and multiply
+ * the fp32 sums by g[e]; the activation limits of the W4A16 range note above
+ * (fp16 x and h, swiglu_limit) hold as stated there. */
 
 /* Human-readable name of a status.  Never NULL. */
 MOE_API const char* moe_status_string(moe_status status);
@@ -209,9 +209,9 @@ MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* topk_ids,
  * W4A16_GEMV_MODULE) when there are fewer than 32 routed rows per expert on
  * average, else a grouped tensor-core GEMM that dequantises the int4 codes
  * into fp16 tiles in shared memory ([glm5next] MOE_GROUPED_MODULE).
- * MOE_W_NVFP4 weights always run that grouped tensor-core GEMM, with E2M1
- * codes and E4M3 block scales decoded into the fp16 tiles.  Every format
- * rounds h to bf16 as the bf16 path does.
+ * MOE_W_NVFP4 weights take the same two kernels by the same rule, decoding
+ * E2M1 codes and E4M3 block scales (in registers, or into the fp16 tiles).
+ * Every format rounds h to bf16 as the bf16 path does.
  * When x_shared != NULL the shared expert runs in the same launches:
  *   shared_out[t] = bf16( SwiGLU_clamped FFN_shared(x_shared[t]) ), unscaled.
  *   x_perm          bf16 [T*k, H]    expert_offsets int32 [E+1]

@@ -65,10 +65,14 @@ PREFILL_W4A16 = LayerConfig("prefill_w4a16", T=16384, H=6144, E=256, k=8, I=2048
                             I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
                             w4a16=True)
 
-# Not one of the five benchmark layers either: the same shape with NVFP4
-# expert weights (the routed NVFP4 MoE the module summary names).
+# Not benchmark layers either: the decode and the large prefill shapes with
+# NVFP4 expert weights (the routed NVFP4 MoE the module summary names).
+DECODE_NVFP4 = LayerConfig("decode_nvfp4", T=32, H=6144, E=256, k=8, I=2048,
+                           I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
+                           nvfp4=True)
 PREFILL_NVFP4 = LayerConfig("prefill_nvfp4", T=16384, H=6144, E=256, k=8, I=2048,
                             I_s=2048, alpha=2.5, renorm=True, bias_range=0.05,
                             nvfp4=True)
 
-CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16, PREFILL_W4A16, PREFILL_NVFP4)}
+CONFIGS = {c.name: c for c in (TINY, MID, LARGE, SKEWED, DECODE_W4A16, PREFILL_W4A16, DECODE_NVFP4,
+                               PREFILL_NVFP4)}

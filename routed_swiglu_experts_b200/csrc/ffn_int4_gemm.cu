@@ -165,37 +165,16 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
   return r;
 }
 
-// One word of FP4 E2M1 codes (k = 0..7 of an aligned 8, low nibble = even k)
-// -> four fp16x2 weights in the same {k0, k4}, {k1, k5}, {k2, k6}, {k3, k7}
-// order as dequant_word, each times its block's E4M3 scale s2 = (s, s).  The
-// nibbles are first regrouped into the bytes k0|k4<<4, k2|k6<<4 (lo) and
-// k1|k5<<4, k3|k7<<4 (hi), so that each conversion (one E2M1 byte -> an
-// fp16 pair, low nibble in the low half) yields a finished pair.  Every
-// product is exact in fp16 (see the file comment).
+// One word of FP4 E2M1 codes -> four fp16x2 weights in the same {k0, k4},
+// {k1, k5}, {k2, k6}, {k3, k7} order as dequant_word (e2m1_word_pairs),
+// each times its block's E4M3 scale s2 = (s, s).  Every product is exact in
+// fp16 (see the file comment).
 __device__ __forceinline__ uint4 dequant_word_fp4(uint32_t w, uint32_t s2) {
-  const uint32_t lo = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
-  const uint32_t hi = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
-  uint4 r;
-  asm("{\n\t.reg .b8 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
-      "mov.b32 {a0, a1, a2, a3}, %4;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %5;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, a0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, a1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b1;\n\t}"
-      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-      : "r"(lo), "r"(hi));
+  uint4 r = e2m1_word_pairs(w);
   r.x = hmul2_u(r.x, s2);  // k0, k4
   r.y = hmul2_u(r.y, s2);  // k1, k5
   r.z = hmul2_u(r.z, s2);  // k2, k6
   r.w = hmul2_u(r.w, s2);  // k3, k7
-  return r;
-}
-
-// Two E4M3 scale bytes (low byte -> low half) to an fp16 pair.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(unsigned short v) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
 }
 

@@ -108,9 +108,8 @@ moe_status check_router_weights(const moe_weights* w) {
 // kernels' own loads.  cfg.num_experts is the number of experts this call
 // computes (0 allowed: shared expert only), `offsets` their [E + 1] row
 // offsets (absolute permuted rows), and w's routed weights hold exactly those
-// experts; e_total is the router's expert count (the int4 path picks its
-// kernel by the average routed rows per expert, R / e_total; NVFP4 experts
-// always take the grouped tensor-core kernel).
+// experts; e_total is the router's expert count (the 4-bit paths pick their
+// kernel by the average routed rows per expert, R / e_total).
 moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_rows, const int32_t* gather_src,
                    const int32_t* offsets, const float* w_perm, int32_t T, void* y_perm, const void* x_shared,
                    void* shared_out, void* ws, const WsLayout& L, cudaStream_t stream, int e_total) {
@@ -128,8 +127,8 @@ moe_status run_ffn(const moe_config& cfg, const moe_weights& w, const void* x_ro
   // few tokens: the shared expert streams its weights with the split-K
   // kernels -- or, beside the int4 GEMVs, inside their launches; otherwise it
   // is one more problem of the tcgen05 launches
-  const bool prefill_path = is_nvfp4(cfg) || (is_int4(cfg) && int4_prefill_preferred(R, e_total));
-  const bool gemv_path = is_int4(cfg) && !prefill_path;
+  const bool prefill_path = is_4bit(cfg) && int4_prefill_preferred(R, e_total);
+  const bool gemv_path = is_4bit(cfg) && !prefill_path;
   const bool shared_in_gemv = with_shared && gemv_path && w4a16_shared_fusable(T, Is);
   const bool shared_small = with_shared && !shared_in_gemv && dense_small_ok(T, H, Is);
   const bool shared_tc = with_shared && !shared_in_gemv && !shared_small;
@@ -229,15 +228,14 @@ WsLayout ws_layout(const moe_config& cfg, int Tmax) {
   L.w_perm = take(R * sizeof(float));
   L.block_base = take(static_cast<size_t>(perm_blocks(static_cast<int>(R))) * E * sizeof(int32_t));
   L.local_rank = take(R * sizeof(int32_t));
-  const bool int4 = cfg.expert_format == MOE_W_INT4_G128;
-  const bool four = int4 || cfg.expert_format == MOE_W_NVFP4;
+  const bool four = cfg.expert_format == MOE_W_INT4_G128 || cfg.expert_format == MOE_W_NVFP4;
   // bf16 experts: the forward gathers the routed rows into x_perm (tiled TMA
   // copies then feed the tensor cores); 4-bit experts gather while converting
   L.x_perm = take(four ? 0 : R * H * 2);
-  // bf16 h, the 4-bit grouped GEMMs' fp16 h [R, I], or the int4 GEMVs' fp32
+  // bf16 h, the 4-bit grouped GEMMs' fp16 h [R, I], or the 4-bit GEMVs' fp32
   // gate/up [R, 2I] (taken only below kInt4PrefillRowsPerExpert rows per expert)
   const size_t r_gemv = std::min(R, static_cast<size_t>(kInt4PrefillRowsPerExpert) * E);
-  L.h = take(int4 ? std::max(R * I * 2, r_gemv * 2 * I * 4) : R * I * 2);
+  L.h = take(four ? std::max(R * I * 2, r_gemv * 2 * I * 4) : R * I * 2);
   L.h_shared = take(T * Is * 2);
   L.y_perm = take(R * H * 2);
   L.shared_out = take(T * H * 2);

@@ -41,6 +41,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
+// NVFP4 element decoding (sm_100a conversions).  One 32-bit word of FP4 E2M1
+// codes (k = 0..7 of an aligned 8, low nibble = even k) -> the exact fp16
+// pairs {k0, k4}, {k1, k5}, {k2, k6}, {k3, k7} in .x, .y, .z, .w.  Three
+// shifts and two LOP3 regroup the nibbles into the bytes k0|k4<<4, k2|k6<<4
+// (lo) and k1|k5<<4, k3|k7<<4 (hi), so that each cvt.rn.f16x2.e2m1x2 (one
+// byte -> a pair, its low nibble into the low half) yields a finished pair.
+__device__ __forceinline__ uint4 e2m1_word_pairs(uint32_t w) {
+  const uint32_t lo = (w & 0x0F0Fu) | ((w >> 12) & 0xF0F0u);
+  const uint32_t hi = ((w >> 4) & 0x0F0Fu) | ((w >> 16) & 0xF0F0u);
+  uint4 r;
+  asm("{\n\t.reg .b8 a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+      "mov.b32 {a0, a1, a2, a3}, %4;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %5;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, a0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, a1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b1;\n\t}"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "r"(lo), "r"(hi));
+  return r;
+}
+
+// Two FP8 E4M3 bytes (low byte -> low half) to an exact fp16 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(unsigned short v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

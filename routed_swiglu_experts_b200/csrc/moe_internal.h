@@ -110,7 +110,8 @@ cudaError_t launch_gemm_gateup(const FfnProblem* routed, const FfnProblem* share
 cudaError_t launch_gemm_down(const FfnProblem* routed, const FfnProblem* shared, int32_t* err, int32_t* queue,
                              int num_sms, cudaStream_t stream);
 
-// W4A16 routed expert kernels (dequantise in registers).
+// 4-bit routed expert GEMVs (dequantise in registers): W4A16 int4 or NVFP4
+// weights, by cfg.expert_format.
 // act16: scratch for the activations in MMA slot order (fp16, [rows, K]).
 // With x_shared != NULL (T <= kW4a16SharedMaxTokens tokens) the shared
 // expert's bf16 projections run in the same two launches: gate/up into
@@ -127,10 +128,10 @@ cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const
                               int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
                               int T, void* h_shared, void* shared_out, cudaStream_t stream);
 
-// 4-bit grouped GEMMs: int4 (W4A16, for many tokens per expert: at least
-// kInt4PrefillRowsPerExpert routed rows per expert on average) or NVFP4 (at
-// every token count) codes dequantised to fp16 in shared memory and fed to
-// the CTA-pair tensor-core pipeline; cfg.expert_format picks the decoder.
+// 4-bit grouped GEMMs for many tokens per expert (at least
+// kInt4PrefillRowsPerExpert routed rows per expert on average): int4 (W4A16)
+// or NVFP4 codes dequantised to fp16 in shared memory and fed to the CTA-pair
+// tensor-core pipeline; cfg.expert_format picks the decoder.
 // tokens16: scratch [rows, H] fp16; h16: scratch [rows, I] fp16; queues:
 // four tile-queue words in the workspace header (gate/up, then down).
 constexpr int kInt4PrefillRowsPerExpert = 32;

@@ -29,6 +29,17 @@
 // fp16 (x/16 in the slots of the 16-times codes: an exact power-of-two
 // scaling), so each group's MMA sum is exactly sum_k (q_k - 8) x_k up to the
 // fp32 accumulation; it is then multiplied by the group's bf16 scale.
+//
+// NVFP4 experts (FP4 E2M1 codes packed the same way, an FP8 E4M3 scale per
+// 16 of K, an fp32 scale per expert tensor) run the same kernels with
+// FP4 = true.  A thread's 32 k of a group are two whole 16-wide scale
+// blocks, and in each MMA its slots hold k of one block only, so it decodes
+// a word into the same slot pairs (e2m1_word_pairs: {k0, k4}, {k1, k5},
+// {k2, k6}, {k3, k7}, no 16-times pairs, activations not divided by 16) and
+// multiplies them by its row's block scale before the MMA -- exact in fp16
+// (e2m1 * e4m3: at most 6 significant bits, magnitude 0 or within
+// [2^-10, 2688]).  The MMAs then accumulate across groups directly, and the
+// tensor scale multiplies the fp32 sum at the store.
 #include <cuda_fp16.h>
 
 #include "moe_internal.h"
@@ -97,14 +108,36 @@ __device__ __forceinline__ void tile_group(float (&t)[4], const uint4 c0, const 
   }
 }
 
+// NVFP4: one 128-wide group of one m16 tile, accumulating into d.  The
+// weights of rows g and g + 8 are decoded and multiplied by their E4M3 block
+// scales (sa*, sb*: (s, s) of the thread's first and second 16 of k) before
+// the MMAs, so no per-group scale follows.
+__device__ __forceinline__ void tile_group_fp4(float (&d)[4], const uint4 c0, const uint4 c8, const uint4 (&act)[4],
+                                               uint32_t sa0, uint32_t sb0, uint32_t sa8, uint32_t sb8) {
+  const uint32_t r0[4] = {c0.x, c0.y, c0.z, c0.w};
+  const uint32_t r8[4] = {c8.x, c8.y, c8.z, c8.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t s0 = i < 2 ? sa0 : sb0, s8 = i < 2 ? sa8 : sb8;
+    const uint4 a = e2m1_word_pairs(r0[i]);
+    const uint4 b = e2m1_word_pairs(r8[i]);
+    mma_f16_16816(d, hmul2_bits(a.x, s0), hmul2_bits(b.x, s8), hmul2_bits(a.y, s0), hmul2_bits(b.y, s8), act[i].x,
+                  act[i].y);
+    mma_f16_16816(d, hmul2_bits(a.z, s0), hmul2_bits(b.z, s8), hmul2_bits(a.w, s0), hmul2_bits(b.w, s8), act[i].z,
+                  act[i].w);
+  }
+}
+
 // Activations in MMA slot order.  One block per row, one thread per 8
 // consecutive values: in {x0..x7} -> out fp16 {x0, x4, x1/16, x5/16, x2, x6,
-// x3/16, x7/16}.  gsrc != NULL: row r of the output is token row
-// gsrc[r] / gk of act (the permutation's gather, done here instead of in a
-// separate copy).
+// x3/16, x7/16} (NVFP4, FP4 = true: {x0, x4, x1, x5, x2, x6, x3, x7}).
+// gsrc != NULL: row r of the output is token row gsrc[r] / gk of act (the
+// permutation's gather, done here instead of in a separate copy).
+template <bool FP4>
 __global__ void __launch_bounds__(128)
     w4a16_prep_kernel(const __nv_bfloat16* __restrict__ act, int k8, const int32_t* __restrict__ gsrc, int gk,
                       uint4* __restrict__ act16) {
+  constexpr float m = FP4 ? 1.f : 0.0625f;  // weight of the odd slots
   const int r = blockIdx.x;
   const int in_row = gsrc != nullptr ? __ldg(gsrc + r) / gk : r;
   const uint4* in = reinterpret_cast<const uint4*>(act) + static_cast<size_t>(in_row) * k8;
@@ -112,9 +145,9 @@ __global__ void __launch_bounds__(128)
   for (int c = threadIdx.x; c < k8; c += blockDim.x) {
     const uint4 v = __ldg(in + c);
     const __half2 a04 = __floats2half2_rn(bf16lo(v.x), bf16lo(v.z));
-    const __half2 b15 = __floats2half2_rn(bf16hi(v.x) * 0.0625f, bf16hi(v.z) * 0.0625f);
+    const __half2 b15 = __floats2half2_rn(bf16hi(v.x) * m, bf16hi(v.z) * m);
     const __half2 a26 = __floats2half2_rn(bf16lo(v.y), bf16lo(v.w));
-    const __half2 b37 = __floats2half2_rn(bf16hi(v.y) * 0.0625f, bf16hi(v.w) * 0.0625f);
+    const __half2 b37 = __floats2half2_rn(bf16hi(v.y) * m, bf16hi(v.w) * m);
     uint4 o;
     o.x = *reinterpret_cast<const uint32_t*>(&a04);
     o.y = *reinterpret_cast<const uint32_t*>(&b15);
@@ -138,9 +171,11 @@ __device__ __forceinline__ float swiglu_clamped_f(float g, float u, float L) {
   return __fdividef(gc, 1.f + __expf(-gc)) * uc;
 }
 
+template <bool FP4>
 __global__ void __launch_bounds__(256)
     w4a16_prep_swiglu_kernel(const float* __restrict__ gu, int I, long long n8, float L, uint4* __restrict__ act16,
                              const float* __restrict__ gus, int Is, long long n8s, __nv_bfloat16* __restrict__ hs) {
+  constexpr float m = FP4 ? 1.f : 0.0625f;  // weight of the odd slots (see w4a16_prep_kernel)
   long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n8) {
     idx -= n8;
@@ -172,9 +207,9 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int j = 0; j < 8; ++j) h[j] = __bfloat162float(__float2bfloat16_rn(swiglu_clamped_f(gv[j], uv[j], L)));
   const __half2 a04 = __floats2half2_rn(h[0], h[4]);
-  const __half2 b15 = __floats2half2_rn(h[1] * 0.0625f, h[5] * 0.0625f);
+  const __half2 b15 = __floats2half2_rn(h[1] * m, h[5] * m);
   const __half2 a26 = __floats2half2_rn(h[2], h[6]);
-  const __half2 b37 = __floats2half2_rn(h[3] * 0.0625f, h[7] * 0.0625f);
+  const __half2 b37 = __floats2half2_rn(h[3] * m, h[7] * m);
   uint4 o;
   o.x = *reinterpret_cast<const uint32_t*>(&a04);
   o.y = *reinterpret_cast<const uint32_t*>(&b15);
@@ -292,11 +327,12 @@ constexpr int kGemvBlocksPerSm = 7;
 constexpr size_t kGemvSmem = static_cast<size_t>(kGemvWarps) * kGemvStages * 64 * sizeof(uint4);
 static_assert(8 % kGemvStages == 0, "ring slots repeat within a batch of 8 groups");
 
-template <bool F32OUT>
+template <bool F32OUT, bool FP4>
 __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
     w4a16_gemv_kernel(const uint4* __restrict__ act16, const int32_t* __restrict__ offsets,
-                      const uint8_t* __restrict__ q, const __nv_bfloat16* __restrict__ scales, int N, int K,
-                      const float* __restrict__ w_perm, void* __restrict__ out, const SharedJob sj) {
+                      const uint8_t* __restrict__ q, const void* __restrict__ scales,
+                      const float* __restrict__ tscale, int N, int K, const float* __restrict__ w_perm,
+                      void* __restrict__ out, const SharedJob sj) {
   extern __shared__ uint4 gemv_ring[];
   constexpr int S = kGemvStages;
   // blocks of the first grid row take the shared expert (when there is one):
@@ -321,8 +357,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
   const size_t row0 = static_cast<size_t>(e) * N + n0 + g;
   const uint8_t* q0 = q + row0 * rb + 16 * t;  // row g; row g + 8 at + q8off
   const uint32_t q8off = 8u * static_cast<uint32_t>(rb);  // < 2^32: a bf16 row of K is < 2^31 bytes
-  const __nv_bfloat16* s0p = scales + row0 * groups;
-  const __nv_bfloat16* s8p = s0p + 8 * groups;
+  // int4: the bf16 scales of rows g and g + 8; NVFP4: their E4M3 block-scale
+  // pairs (blocks 8 q + 2t and + 1 of group q, at 16-bit index 4 q)
+  const __nv_bfloat16* s0p = FP4 ? nullptr : static_cast<const __nv_bfloat16*>(scales) + row0 * groups;
+  const __nv_bfloat16* s8p = FP4 ? nullptr : s0p + 8 * groups;
+  const unsigned short* f0p =
+      FP4 ? reinterpret_cast<const unsigned short*>(static_cast<const uint8_t*>(scales) + row0 * (K / 16)) + t
+          : nullptr;
+  const unsigned short* f8p = FP4 ? f0p + 8 * (K / 32) : nullptr;
+  const float ts = FP4 ? __ldg(tscale + e) : 1.f;
   uint4* ring = gemv_ring + warp * S * 64 + lane;
   // codes of group i (rows g and g + 8, 16 bytes each) from base qb into ring slot `slot`
   auto issue = [&](const uint8_t* qb, int i, int slot) {
@@ -356,13 +399,19 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
           cp_async_commit();
           const uint4* st = ring + (jj % S) * 64;
           const uint4 c0 = st[0], c8 = st[32];
-          float tt[4];
-          tile_group(tt, c0, c8, act);
-          const float a0 = __bfloat162float(__ldg(s0p + gq)), a8 = __bfloat162float(__ldg(s8p + gq));
-          acc[0] = fmaf(a0, tt[0], acc[0]);
-          acc[1] = fmaf(a0, tt[1], acc[1]);
-          acc[2] = fmaf(a8, tt[2], acc[2]);
-          acc[3] = fmaf(a8, tt[3], acc[3]);
+          if (FP4) {
+            const uint32_t v0 = e4m3x2_to_f16x2(__ldg(f0p + 4 * gq)), v8 = e4m3x2_to_f16x2(__ldg(f8p + 4 * gq));
+            tile_group_fp4(acc, c0, c8, act, __byte_perm(v0, 0, 0x1010), __byte_perm(v0, 0, 0x3232),
+                           __byte_perm(v8, 0, 0x1010), __byte_perm(v8, 0, 0x3232));
+          } else {
+            float tt[4];
+            tile_group(tt, c0, c8, act);
+            const float a0 = __bfloat162float(__ldg(s0p + gq)), a8 = __bfloat162float(__ldg(s8p + gq));
+            acc[0] = fmaf(a0, tt[0], acc[0]);
+            acc[1] = fmaf(a0, tt[1], acc[1]);
+            acc[2] = fmaf(a8, tt[2], acc[2]);
+            acc[3] = fmaf(a8, tt[3], acc[3]);
+          }
         }
       }
     }
@@ -374,10 +423,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
       const int col = n0 + g + 8 * (cc >> 1);
       if (tok < ntok) {
         const int r = tc + tok;
+        const float a = FP4 ? acc[cc] * ts : acc[cc];
         if (F32OUT) {
-          static_cast<float*>(out)[static_cast<size_t>(r) * N + col] = acc[cc];
+          static_cast<float*>(out)[static_cast<size_t>(r) * N + col] = a;
         } else {
-          const float v = acc[cc] * (w_perm != nullptr ? w_perm[r] : 1.f);
+          const float v = a * (w_perm != nullptr ? w_perm[r] : 1.f);
           static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(r) * N + col] = __float2bfloat16_rn(v);
         }
       }
@@ -385,23 +435,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kGemvBlocksPerSm)
   }
 }
 
+template <bool FP4>
 cudaError_t launch_prep(const void* act, int rows, int K, const int32_t* gsrc, int gk, void* act16,
                         cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  return launch_kernel(w4a16_prep_kernel, dim3(rows), dim3(128), 0, stream,
+  return launch_kernel(w4a16_prep_kernel<FP4>, dim3(rows), dim3(128), 0, stream,
                                static_cast<const __nv_bfloat16*>(act), K / 8, gsrc, gk, static_cast<uint4*>(act16));
 }
 
-template <bool F32OUT>
-cudaError_t launch_gemv(const void* q, const void* scales, int E, int N, int K, const void* act16,
-                        const int32_t* offsets, const float* w_perm, void* out, const SharedJob& sj,
-                        cudaStream_t stream) {
+template <bool F32OUT, bool FP4>
+cudaError_t launch_gemv(const void* q, const void* scales, const float* tscale, int E, int N, int K,
+                        const void* act16, const int32_t* offsets, const float* w_perm, void* out,
+                        const SharedJob& sj, cudaStream_t stream) {
   const int nx = std::max(N, sj.w != nullptr ? sj.N : 0);
   const dim3 grid((nx + kGemvRows - 1) / kGemvRows, E + (sj.w != nullptr ? 1 : 0));
   if (grid.y == 0) return cudaSuccess;  // no routed expert and no shared expert in this call
-  return launch_kernel(w4a16_gemv_kernel<F32OUT>, grid, dim3(kGemvWarps * 32), kGemvSmem, stream,
-                               static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q),
-                               static_cast<const __nv_bfloat16*>(scales), N, K, w_perm, out, sj);
+  return launch_kernel(w4a16_gemv_kernel<F32OUT, FP4>, grid, dim3(kGemvWarps * 32), kGemvSmem, stream,
+                       static_cast<const uint4*>(act16), offsets, static_cast<const uint8_t*>(q), scales, tscale, N,
+                       K, w_perm, out, sj);
 }
 
 }  // namespace
@@ -412,34 +463,45 @@ cudaError_t launch_w4a16_gateup(const moe_config& cfg, const moe_weights& w, con
                                 const int32_t* gather_src, const int32_t* offsets, int rows, void* act16, float* gu,
                                 const void* x_shared, int T, float* gu_shared, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts;
-  cudaError_t e = launch_prep(x_rows, rows, H, gather_src, cfg.top_k, act16, stream);
+  const bool fp4 = cfg.expert_format == MOE_W_NVFP4;
+  cudaError_t e = fp4 ? launch_prep<true>(x_rows, rows, H, gather_src, cfg.top_k, act16, stream)
+                      : launch_prep<false>(x_rows, rows, H, gather_src, cfg.top_k, act16, stream);
   if (e != cudaSuccess) return e;
   SharedJob sj{};
   if (x_shared != nullptr)  // shared gate/up [2 I_s, H] x tokens [T, H] -> fp32 [T, 2 I_s]
     sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_gate_up), static_cast<const __nv_bfloat16*>(x_shared),
                    gu_shared, 2 * cfg.shared_inter, H, T};
   // W_gu [E, 2I, H/2]: one matrix of 2I rows per expert (gate rows, then up rows)
-  return launch_gemv<true>(w.w_gate_up, w.s_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu, sj, stream);
+  if (fp4)
+    return launch_gemv<true, true>(w.w_gate_up, w.s_gate_up, w.g_gate_up, E, 2 * I, H, act16, offsets, nullptr, gu,
+                                   sj, stream);
+  return launch_gemv<true, false>(w.w_gate_up, w.s_gate_up, nullptr, E, 2 * I, H, act16, offsets, nullptr, gu, sj,
+                                  stream);
 }
 
 cudaError_t launch_w4a16_down(const moe_config& cfg, const moe_weights& w, const float* gu, const int32_t* offsets,
                               int rows, void* act16, const float* w_perm, void* y_perm, const float* gu_shared,
                               int T, void* h_shared, void* shared_out, cudaStream_t stream) {
   const int I = cfg.expert_inter, H = cfg.hidden, E = cfg.num_experts, Is = cfg.shared_inter;
+  const bool fp4 = cfg.expert_format == MOE_W_NVFP4;
   const long long n8 = static_cast<long long>(rows) * (I / 8);
   const long long n8s = gu_shared != nullptr ? static_cast<long long>(T) * (Is / 8) : 0;
   if (n8 + n8s > 0) {
-    cudaError_t e = launch_kernel(w4a16_prep_swiglu_kernel, dim3(static_cast<unsigned>((n8 + n8s + 255) / 256)),
-                                          dim3(256), 0, stream, gu, I, n8, cfg.swiglu_limit,
-                                          static_cast<uint4*>(act16), gu_shared, Is, n8s,
-                                          static_cast<__nv_bfloat16*>(h_shared));
+    const dim3 grid(static_cast<unsigned>((n8 + n8s + 255) / 256));
+    cudaError_t e =
+        fp4 ? launch_kernel(w4a16_prep_swiglu_kernel<true>, grid, dim3(256), 0, stream, gu, I, n8, cfg.swiglu_limit,
+                            static_cast<uint4*>(act16), gu_shared, Is, n8s, static_cast<__nv_bfloat16*>(h_shared))
+            : launch_kernel(w4a16_prep_swiglu_kernel<false>, grid, dim3(256), 0, stream, gu, I, n8, cfg.swiglu_limit,
+                            static_cast<uint4*>(act16), gu_shared, Is, n8s, static_cast<__nv_bfloat16*>(h_shared));
     if (e != cudaSuccess) return e;
   }
   SharedJob sj{};
   if (gu_shared != nullptr)  // shared down [H, I_s] x h_s [T, I_s] -> bf16 [T, H], unscaled
     sj = SharedJob{static_cast<const __nv_bfloat16*>(w.shared_w_down), static_cast<const __nv_bfloat16*>(h_shared),
                    shared_out, H, Is, T};
-  return launch_gemv<false>(w.w_down, w.s_down, E, H, I, act16, offsets, w_perm, y_perm, sj, stream);
+  if (fp4)
+    return launch_gemv<false, true>(w.w_down, w.s_down, w.g_down, E, H, I, act16, offsets, w_perm, y_perm, sj, stream);
+  return launch_gemv<false, false>(w.w_down, w.s_down, nullptr, E, H, I, act16, offsets, w_perm, y_perm, sj, stream);
 }
 
 }  // namespace moe

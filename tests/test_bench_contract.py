@@ -37,7 +37,8 @@ def test_gemm_flops_of_the_mid_layer():
     # ... + token prep + dequantising gate/up and down + bf16 shared gate/up
     # and down launches
     ("prefill_w4a16", 11),
-    # NVFP4 experts take the same grouped kernels at every token count
+    # NVFP4 experts take the same two paths by the same rule
+    ("decode_nvfp4", 10),
     ("prefill_nvfp4", 11),
 ])
 def test_launches_per_step_match_the_launch_lists(name, expected):
@@ -68,6 +69,17 @@ def test_w4a16_bytes_of_one_touched_expert():
     assert touched == 1
     assert codes + scales == 19_464_192
     assert total == codes + scales + shared + acts
+
+
+def test_nvfp4_bytes_of_one_touched_expert():
+    import torch
+    cfg = CONFIGS["decode_nvfp4"]
+    touched, total = bench.w4a16_bytes(cfg, torch.tensor([[7, 7]]))
+    H, I, Is, T, k = 6144, 2048, 2048, cfg.T, cfg.k
+    codes = (2 * I * H + H * I) // 2            # two E2M1 codes per byte
+    scales = (2 * I * H + H * I) // 16          # one E4M3 byte per 16 weights
+    assert touched == 1
+    assert total == codes + scales + 8 + 2 * (3 * H * Is) + 2 * T * H * (2 + 2 * k)
 
 
 def test_traffic_is_reported_only_for_the_profiled_source(tmp_path, monkeypatch):

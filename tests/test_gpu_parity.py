@@ -67,12 +67,17 @@ EDGE = {
                                     swiglu_limit=255.0, x_scale=50.0, w4a16=True),
     "w4a16_prefill_wide_limit": LayerConfig("w4a16_prefill_wide_limit", T=300, H=256, E=4, k=2, I=256,
                                             I_s=128, swiglu_limit=255.0, x_scale=50.0, w4a16=True),
-    # NVFP4 experts (grouped tensor-core GEMM at every token count): few tokens
-    # (shared expert on the split-K path), several token and weight tiles with
-    # ragged tails (K = 384: the second code copy half past the row), many
-    # tiles per expert, the clamp, and the widest clamp with large activations
+    # NVFP4 experts.  Fewer than 32 rows per expert: the register-dequant GEMV
+    # (shared expert in its launches), with several 8-token chunks per expert,
+    # and at the widest clamp with large activations.  32 or more: the grouped
+    # tensor-core GEMM over several token and weight tiles with ragged tails
+    # (K = 384: the second code copy half past the row), many tiles per
+    # expert, the clamp, and the widest clamp with large activations
     "nvfp4_small": LayerConfig("nvfp4_small", T=20, H=256, E=6, k=2, I=128, I_s=128, alpha=2.5, renorm=True,
                                bias_range=0.05, nvfp4=True),
+    "nvfp4_chunks": LayerConfig("nvfp4_chunks", T=40, H=384, E=8, k=2, I=256, I_s=0, nvfp4=True),
+    "nvfp4_gemv_wide_limit": LayerConfig("nvfp4_gemv_wide_limit", T=20, H=256, E=6, k=2, I=128, I_s=128,
+                                         swiglu_limit=255.0, x_scale=50.0, nvfp4=True),
     "nvfp4_prefill": LayerConfig("nvfp4_prefill", T=700, H=512, E=8, k=2, I=384, I_s=256, alpha=2.5, renorm=True,
                                  bias_range=0.05, nvfp4=True),
     "nvfp4_wide": LayerConfig("nvfp4_wide", T=1500, H=1024, E=16, k=4, I=640, I_s=384, alpha=2.5, renorm=True,
@@ -244,13 +249,15 @@ def test_forward_replays_from_a_cuda_graph(small_inputs, name):
     del graph
 
 
-def test_nvfp4_every_scale_byte():
+@pytest.mark.parametrize("T", [300, 16])
+def test_nvfp4_every_scale_byte(T):
     """The down weight's E4M3 block scales vary by output row and take every
     finite E4M3 pattern (both signs, the subnormals, 448): output column n of
     y_perm is one scale value times an unscaled sum, so each column is
     compared with the oracle's on its own.  The E4M3 NaN patterns are left
-    out (they make NaN weights by definition)."""
-    cfg = LayerConfig("nvfp4_scales", T=300, H=256, E=2, k=1, I=128, I_s=0, nvfp4=True)
+    out (they make NaN weights by definition).  T = 300: the grouped GEMM;
+    T = 16 (8 rows per expert): the GEMV."""
+    cfg = LayerConfig("nvfp4_scales", T=T, H=256, E=2, k=1, I=128, I_s=0, nvfp4=True)
     inp = moe_inputs.make_layer(cfg, seed=5)
     finite = [b for b in range(256) if b not in (0x7F, 0xFF)] + [0x38, 0xB8]   # 256 rows
     rows = torch.tensor(finite, dtype=torch.int64).to(torch.uint8)
@@ -284,9 +291,9 @@ def test_tied_router_prefers_lower_id(small_inputs, name):
 
 # ------------------------------------------------------ benchmark layers ----
 
-FULL = ["mid", "skewed", "large_prefill", "decode_w4a16", "prefill_w4a16"]
+FULL = ["mid", "skewed", "large_prefill", "decode_w4a16", "prefill_w4a16", "decode_nvfp4"]
 # layers whose every output row is compared (the oracle runs them in seconds)
-ALL_ROWS = {"mid", "decode_w4a16"}
+ALL_ROWS = {"mid", "decode_w4a16", "decode_nvfp4"}
 TILE_ROWS = 256         # routed rows per token tile of the grouped GEMMs (a CTA pair)
 MIN_SAMPLE = 1024       # tokens compared on the other layers, at least
 
