@@ -269,3 +269,42 @@ def test_forward_ep_argument_checks(lib):
     # local experts need weights, an empty range does not
     assert _call_ep(lib, cfg, _fake_weights(w_gate_up=None), 0, 4) == _abi.MOE_ERR_INVALID_ARG
     assert _call_ep(lib, cfg, _fake_weights(w_gate_up=None, w_down=None), 4, 4, T=0) == _abi.MOE_OK
+
+
+def test_header_is_plain_c_and_matches_the_binding(tmp_path):
+    """include/moe.h compiles as C99 on its own (no CUDA headers), and the
+    struct layouts, enum values and limits it declares are the ones the
+    ctypes binding mirrors."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"moe_config": _abi.moe_config, "moe_weights": _abi.moe_weights}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "moe.h"', "int main(void) {"]
+    for sname, ct in structs.items():
+        lines.append(f'  printf("sizeof {sname} %zu\\n", sizeof({sname}));')
+        for f, _ in ct._fields_:
+            lines.append(f'  printf("offset {sname}.{f} %zu\\n", offsetof({sname}, {f}));')
+    consts = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA",
+              "MOE_ERR_DEVICE_TIMEOUT", "MOE_W_BF16", "MOE_W_INT4_G128", "MOE_W_NVFP4", "MOE_MAX_TOP_K",
+              "MOE_MAX_EXPERTS", "MOE_NO_ALLOC_MAX_ROWS", "MOE_SELFTEST_SCRATCH_BYTES", "MOE_SELFTEST_PAIR_BF16",
+              "MOE_SELFTEST_PAIR_INT4"]
+    for c in consts:
+        lines.append(f'  printf("const {c} %ld\\n", (long)({c}));')
+    lines.append('  printf("const MOE_INT4_MAX_SWIGLU_LIMIT %.1f\\n", (double)MOE_INT4_MAX_SWIGLU_LIMIT);')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe)], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {" ".join(l.split()[:2]): l.split()[2] for l in out if l}
+    for sname, ct in structs.items():
+        assert int(got[f"sizeof {sname}"]) == ctypes.sizeof(ct), sname
+        for f, _ in ct._fields_:
+            assert int(got[f"offset {sname}.{f}"]) == getattr(ct, f).offset, f"{sname}.{f}"
+    for c in consts:
+        assert int(got[f"const {c}"]) == getattr(_abi, c), c
+    assert float(got["const MOE_INT4_MAX_SWIGLU_LIMIT"]) == _abi.MOE_INT4_MAX_SWIGLU_LIMIT
