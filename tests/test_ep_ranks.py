@@ -53,6 +53,28 @@ def test_local_tensors_slice_the_right_rows():
     # gate rows of the slice, then its up rows (gate = shard 0, up = shard 1 of the fused weight)
     assert torch.equal(loc["shared_w_gate_up"], torch.cat([sgu[16:24], sgu[24 + 16:24 + 24]]))
     assert torch.equal(loc["shared_w_down"], sd[:, 16:24])
+    assert loc["s_gate_up"] is None and loc["g_gate_up"] is None and loc["g_down"] is None
+
+
+def test_local_tensors_slice_the_4bit_scales_with_their_experts():
+    """Block scales and (NVFP4) per-expert tensor scales follow the rank's
+    expert range like the codes they belong to."""
+    E, I, H = 5, 16, 32
+    q_gu = torch.arange(E * 2 * I * H // 2).reshape(E, 2 * I, H // 2)
+    q_d = torch.arange(E * H * I // 2).reshape(E, H, I // 2)
+    s_gu = torch.arange(E * 2 * I * H // 16).reshape(E, 2 * I, H // 16)
+    s_d = torch.arange(E * H * I // 16).reshape(E, H, I // 16)
+    g_gu = torch.arange(E, dtype=torch.float32) + 0.5
+    g_d = torch.arange(E, dtype=torch.float32) + 0.25
+    for rank in range(2):
+        loc = ep.local_tensors(rank, 2, E, 0, w_gate_up=q_gu, w_down=q_d, s_gate_up=s_gu, s_down=s_d,
+                               g_gate_up=g_gu, g_down=g_d)
+        b, e = loc["expert_range"]
+        assert (b, e) == ((0, 3), (3, 5))[rank]
+        for name, full in (("w_gate_up", q_gu), ("w_down", q_d), ("s_gate_up", s_gu), ("s_down", s_d),
+                           ("g_gate_up", g_gu), ("g_down", g_d)):
+            assert torch.equal(loc[name], full[b:e]), name
+            assert loc[name].is_contiguous()
 
 
 def _rank_main(rank, world, port, results):
