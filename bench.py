@@ -721,7 +721,7 @@ def bench_reference(args):
     import oracle
     cfg, inp = make_inputs(args.workload)
     # per-step sample sized so the whole run stays within a few minutes
-    sample = 512
+    sample = min(512, cfg.T)
     t0 = time.perf_counter()
     oracle.moe_forward(inp, tokens=range(sample))
     est = time.perf_counter() - t0

@@ -119,3 +119,20 @@ def test_clock_sampler_drains_a_pipe_larger_than_its_buffer():
     res = c.finish()
     assert time.time() - t0 < 15
     assert res["samples"] == n and res["sm_mhz"] == 1965.0 and res["reasons"] == ["sw_power_cap"]
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    """`bench.py --impl reference` times the oracle on the host (no GPU) and
+    prints one JSON line with the contract's keys, on a layer with fewer
+    tokens than its default per-step sample."""
+    import json
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3", "--workload", "tiny"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "gpu_launches"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["gpu_launches"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert "64 of the 64 tokens" in line["cpu_baseline"]["sample"]
